@@ -1,0 +1,179 @@
+"""CPU oracle of the NVFP4 W4A4 linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` import this package.  The CUDA library never loads it, and it
+shares no code, header, table or constant generator with the CUDA library:
+the arithmetic lives in ``nvfp4_oracle.c`` (plain C, fp32 steps as single IEEE
+operations, float64 for dequantization and the GEMM reference) and this module
+only marshals numpy arrays into it.
+
+Sources (web pages on arXiv 2609.04098, "Why Gated DeltaNet Survives 4-Bit
+Quantization"): the NVFP4 format and the W4A4 product on the ta-paperlens page
+("前提1") and the arxiv-wiki page ("접근 방법"); the fused-group global-scale
+repair on the arxiv-wiki page ("접근 방법", "개발자 관점") and the abstract on the
+shd-paper page.  Readings the pages leave open are listed in the C file's
+header.  Everything except the arithmetic order for non-power-of-two global
+scales is pinned by tests/test_oracle_*.py; that order is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libnvfp4_oracle.so")
+_lib = None
+
+BLOCK = 16
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE fp32, no contraction, OpenMP rows)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+               "-fopenmp", "-o", _LIB_PATH + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        i64, f32, f64, vp, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
+        L.oracle_e2m1_decode.argtypes, L.oracle_e2m1_decode.restype = [i32], f64
+        L.oracle_e4m3_decode.argtypes, L.oracle_e4m3_decode.restype = [i32], f64
+        L.oracle_e2m1_encode.argtypes, L.oracle_e2m1_encode.restype = [f32], i32
+        L.oracle_e4m3_encode.argtypes, L.oracle_e4m3_encode.restype = [f32], i32
+        L.oracle_sf_offset.argtypes, L.oracle_sf_offset.restype = [i64, i64, i64], i64
+        L.oracle_sf_bytes.argtypes, L.oracle_sf_bytes.restype = [i64, i64], i64
+        L.oracle_global_scale.argtypes, L.oracle_global_scale.restype = [vp, i64], f32
+        L.oracle_quantize.argtypes, L.oracle_quantize.restype = [vp, i64, i64, i64, f32, vp, vp, i64], None
+        L.oracle_harmonize.argtypes, L.oracle_harmonize.restype = [vp, i64, i32, vp, vp], f32
+        L.oracle_dequantize.argtypes, L.oracle_dequantize.restype = [vp, vp, i64, i64, f32, i64, vp], None
+        L.oracle_gemm_f64.argtypes, L.oracle_gemm_f64.restype = [vp, vp, i64, i64, i64, f64, vp, vp], None
+        L.oracle_sf_gather.argtypes, L.oracle_sf_gather.restype = [vp, vp, i64, i64, vp], None
+        L.oracle_num_threads.argtypes, L.oracle_num_threads.restype = [], i32
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+# ------------------------------------------------------------------ codecs
+def e2m1_decode(code: int) -> float:
+    return lib().oracle_e2m1_decode(int(code))
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().oracle_e4m3_decode(int(code))
+
+
+def e2m1_encode(y) -> int:
+    return lib().oracle_e2m1_encode(float(np.float32(y)))
+
+
+def e4m3_encode(t) -> int:
+    return lib().oracle_e4m3_encode(float(np.float32(t)))
+
+
+# ------------------------------------------------------------------ layout
+def sf_bytes(rows: int, K: int) -> int:
+    return int(lib().oracle_sf_bytes(rows, K))
+
+
+def sf_offset(r: int, c: int, K: int) -> int:
+    return int(lib().oracle_sf_offset(r, c, K))
+
+
+def sf_gather(sf: np.ndarray, rows, K: int) -> np.ndarray:
+    """Scale bytes of `rows` as a plain [len(rows), K/16] uint8 array."""
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((rows.size, K // BLOCK), dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    lib().oracle_sf_gather(_ptr(sf), _ptr(rows), rows.size, K, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- steps
+def global_scale(x: np.ndarray) -> np.float32:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return np.float32(lib().oracle_global_scale(_ptr(x), x.size))
+
+
+def quantize(x: np.ndarray, g, sf: np.ndarray | None = None, sf_row0: int = 0,
+             sf_rows_total: int | None = None):
+    """Quantize x [rows, K] (float32; bf16 callers convert exactly first).
+
+    Returns (codes [rows, K/2] uint8, sf flat uint8 swizzled buffer)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, K = x.shape
+    assert K % 64 == 0
+    if sf is None:
+        total = rows if sf_rows_total is None else sf_rows_total
+        sf = np.zeros(sf_bytes(total, K), dtype=np.uint8)
+    codes = np.zeros((rows, K // 2), dtype=np.uint8)
+    lib().oracle_quantize(_ptr(x), rows, K, K, float(np.float32(g)), _ptr(codes), _ptr(sf), sf_row0)
+    return codes, sf
+
+
+def harmonize(sf: np.ndarray, K: int, row_offsets, gscales) -> np.float32:
+    """In-place rewrite of a fused group's scales to g* = max(gscales); returns g*."""
+    offs = np.ascontiguousarray(np.asarray(row_offsets, dtype=np.int64))
+    gs = np.ascontiguousarray(np.asarray(gscales, dtype=np.float32))
+    assert offs.size == gs.size + 1
+    return np.float32(lib().oracle_harmonize(_ptr(sf), K, gs.size, _ptr(offs), _ptr(gs)))
+
+
+def dequantize(codes: np.ndarray, sf: np.ndarray, g, sf_row0: int = 0) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((rows, K), dtype=np.float64)
+    lib().oracle_dequantize(_ptr(codes), _ptr(np.ascontiguousarray(sf)), rows, K,
+                            float(np.float32(g)), sf_row0, _ptr(out))
+    return out
+
+
+def gemm_f64(a: np.ndarray, b: np.ndarray, alpha: float, brute: bool = False):
+    """Y = alpha * a @ b.T and Yabs = |alpha| * |a| @ |b|.T in float64.
+
+    brute=True runs the plain C triple loop; otherwise numpy's float64 matmul
+    (a library primitive) computes the same sums."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    b = np.ascontiguousarray(b, dtype=np.float64)
+    M, K = a.shape
+    N = b.shape[0]
+    if brute:
+        y = np.empty((M, N)); yabs = np.empty((M, N))
+        lib().oracle_gemm_f64(_ptr(a), _ptr(b), M, N, K, float(alpha), _ptr(y), _ptr(yabs))
+        return y, yabs
+    y = (a @ b.T) * alpha
+    yabs = (np.abs(a) @ np.abs(b).T) * abs(alpha)
+    return y, yabs
+
+
+def linear_reference(x: np.ndarray, gx, w_codes: np.ndarray, w_sf: np.ndarray, gw,
+                     brute: bool = False):
+    """The whole W4A4 linear on the CPU: quantize x, dequantize both operands,
+    float64 GEMM with alpha = gx*gw.  Returns (y, yabs, x_codes, x_sf)."""
+    xc, xs = quantize(x, gx)
+    # unit-scale operands: every product dec(q)dec(s)dec(q')dec(s') has at most
+    # 12 significant bits, so the float64 sums are exact for these ranges; the
+    # two global scales are applied once, in float64, at the end
+    a = dequantize(xc, xs, 1.0)
+    b = dequantize(w_codes, w_sf, 1.0)
+    y, yabs = gemm_f64(a, b, float(np.float64(gx) * np.float64(gw)), brute=brute)
+    return y, yabs, xc, xs
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
