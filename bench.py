@@ -1,0 +1,458 @@
+#!/usr/bin/env python3
+"""Benchmark of the NVFP4 W4A4 linear layer on B200.
+
+One step = the whole hot path on one batch: NVFP4-quantize the activation
+(nvfp4_quantize) and run the block-scaled W4A4 GEMM against the pre-quantized
+weight (nvfp4_gemm) -- exactly the two launches w4a4_gemm makes -- on the
+prefill MLP gate/up workload (X bf16 [32768, 5120], W [34816, 5120], BF16
+out).  Weights are quantized offline (untimed); the activation global scale is
+a static calibrated scale (untimed), as in the pages' checkpoints.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line.  Under torchrun each rank runs an independent replica
+(the layer is data-parallel over tokens and needs no collective); the time is
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_w4a4_quantized_06_b200 import workloads as W  # noqa: E402
+
+HEADLINE = "prefill_mlp_gate_up"
+METRIC = "W4A4 GEMM TFLOPS (incl. act quantize) & % dense FP4 peak; quantize GB/s"
+FP4_OVER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio on B200
+FP4_SPEC_TFLOPS = 9000.0     # NVIDIA's dense FP4 figure, for context
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clocks and throttle reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
+                                                          if r[3].replace(".", "").isdigit())}
+
+
+# ---------------------------------------------------------------- helpers
+def quantized_weight(wl, dev):
+    """Offline weight preparation: per-module quantize into the fused buffer,
+    then the fused-group global-scale harmonization (untimed)."""
+    from nvfp4_w4a4_quantized_06_b200 import native
+    K, N = wl.K, wl.N
+    offs = np.concatenate([[0], np.cumsum(wl.modules)]).astype(np.int64)
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty(native.sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    gs = []
+    for m in range(len(wl.modules)):
+        wd = W.make_w(wl, m).to(dev)
+        g = native.amax_gscale(wd)
+        native.quantize(wd, g, codes=codes[offs[m]:offs[m + 1]], sf=sf, sf_row0=int(offs[m]), sf_rows_total=N)
+        gs.append(g)
+        del wd
+    gw = native.harmonize(sf, N, K, offs, torch.cat(gs)) if len(gs) > 1 else gs[0]
+    return codes, sf, gw
+
+
+def kernel_src_hash():
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "ptx.cuh", "nvfp4w4a4.cu"):
+        h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_06_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(name)
+    if not d or d.get("src_hash") != kernel_src_hash():
+        return None
+    return d.get("bytes_per_launch")
+
+
+def quant_bytes(M, K):
+    return M * K * 2 + M * K // 2 + ((M + 127) // 128 * 128) * (K // 16)
+
+
+# ------------------------------------------------------------ native arm
+def run_native(args, rank, world, dev):
+    from nvfp4_w4a4_quantized_06_b200 import native
+    wl = W.WORKLOADS[args.workload]
+    M, N, K = wl.M, wl.N, wl.K
+    x_cpu = W.make_x(wl)
+    x = x_cpu.to(dev)
+    w_codes, w_sf, gw = quantized_weight(wl, dev)
+    gx = native.amax_gscale(x)                       # static calibrated activation scale
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    a_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    a_sf = torch.empty(native.sf_bytes(M, K), dtype=torch.uint8, device=dev)
+    ws_bytes = native.lib().nvfp4_gemm_workspace_bytes(M, N, K)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        native.quantize(x, gx, codes=a_codes, sf=a_sf)
+        native.gemm(a_codes, a_sf, gx, w_codes, w_sf, gw, out=y, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = native.launch_count()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        native.quantize(x, gx, codes=a_codes, sf=a_sf)
+        ev[s][1].record(stream)
+        native.gemm(a_codes, a_sf, gx, w_codes, w_sf, gw, out=y, workspace=ws)
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = native.launch_count() - launches0
+    clocks = sampler.stop()
+    flags = native.last_device_status()
+    assert flags == 0, f"device error flags {flags}"
+
+    total_ms = t_start.elapsed_time(t_end)
+    tq = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    tg = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
+    if world > 1:
+        t = torch.tensor([total_ms, sum(tq), sum(tg)], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, sq, sg = t.tolist()
+    else:
+        sq, sg = sum(tq), sum(tg)
+    ms_per_step = total_ms / args.steps
+    flops = 2.0 * M * N * K
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    pk = peaks()
+    tq_ms, tg_ms = sq / args.steps, sg / args.steps
+    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    gemm_tflops = flops / (tg_ms * 1e-3) / 1e12
+    q_gbs = quant_bytes(M, K) / (tq_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public one-call API, host buffers
+    e2e = measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world)
+
+    also = {}
+    if world == 1 and not args.headline_only:
+        also = measure_secondary(native, dev)
+        torch.cuda.empty_cache()
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3/16 x fp32 scale) -> fp32 accumulate -> bf16",
+        "data": "synthetic (seeded PCG64 Gaussians with block outliers; random-init weights)",
+        "config": {"workload": f"{wl.name} {M}x{N}x{K}", "M": M, "N": N, "K": K, "x_dtype": "bf16",
+                   "y_dtype": "bf16", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (X 335 MB, Y 2.28 GB per step; no flush)"},
+        "breakdown_ms": {"quantize": round(tq_ms, 4), "gemm": round(tg_ms, 4)},
+        "quantize_gbs": round(q_gbs, 1),
+        "quantize_frac_hbm": round(q_gbs / pk["hbm_gbs"], 3),
+        "gemm_tflops": round(gemm_tflops, 1),
+        "frac_fp4_spec": round(value / world / FP4_SPEC_TFLOPS, 3),
+        "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256,bf16>",
+                     "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / fp4_peak, 3),
+                     "peak_src": f"{pk['src']} bf16 burst x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
+                     "traffic": recorded_traffic("gemm_prefill_mlp_gate_up")},
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if also:
+        out["also"] = also
+    return out
+
+
+def measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world, steps=3):
+    """Same metric through w4a4_gemm with host buffers: pinned H2D of X, the
+    layer, D2H of Y, all inside the timed region."""
+    x_host = x_cpu.pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x_host, device=dev)
+    y_dev = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(native.linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        native.linear(x_dev, gx, w_codes, w_sf, gw, out=y_dev, workspace=ws)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        one()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.item()
+    del ws, x_dev, y_dev
+    return {"value": round(2.0 * M * N * K * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": x_host.numel() * 2,
+            "d2h_bytes_per_step": y_host.numel() * 2}
+
+
+def measure_secondary(native, dev):
+    """The other workloads of the layer, one line each (median of events):
+    GDN fused groups (TFLOP/s), decode shapes (HBM GB/s over weights+X+Y,
+    rotating over >= 4x L2 of weight copies inside a CUDA graph)."""
+    res = {}
+    pk = peaks()
+    for name in ("gdn_qkv_z", "gdn_gates_ab"):
+        wl = W.WORKLOADS[name]
+        x = W.make_x(wl).to(dev)
+        wc, wsf, gw = quantized_weight(wl, dev)
+        gx = native.amax_gscale(x)
+        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+        flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+        times = []
+        for i in range(12):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            native.linear(x, gx, wc, wsf, gw, out=y, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        byts = wl.M * wl.K * 2 + wl.N * wl.K // 2 + wl.N * wl.K // 16 + wl.M * wl.N * 2
+        res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4),
+                     "tflops": round(wl.flops / (ms * 1e-3) / 1e12, 1),
+                     "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
+                     "l2": "512 MB flush between reps"}
+        del x, wc, wsf, y, ws, flush
+    for name in ("decode_out_proj", "decode_down_proj"):
+        wl = W.WORKLOADS[name]
+        x = W.make_x(wl).to(dev)
+        wc, wsf, gw = quantized_weight(wl, dev)
+        gx = native.amax_gscale(x)
+        wbytes = wc.numel() + wsf.numel()
+        copies = max(4, int(np.ceil(4 * 126e6 / wbytes)))
+        wcs = [wc.clone() for _ in range(copies)]
+        wsfs = [wsf.clone() for _ in range(copies)]
+        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+        for i in range(copies):                   # warm-up outside capture
+            native.linear(x, gx, wcs[i], wsfs[i], gw, out=y, workspace=ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(copies):
+                native.linear(x, gx, wcs[i], wsfs[i], gw, out=y, workspace=ws)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / (reps * copies)
+        byts = wbytes + wl.M * wl.K * 2 + wl.M * wl.N * 2
+        res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "us": round(ms * 1e3, 2),
+                     "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
+                     "l2": f"CUDA graph over {copies} weight copies ({copies * wbytes / 1e6:.0f} MB)"}
+        del g, wcs, wsfs, x, y, ws
+    assert native.last_device_status() == 0
+    return res
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample(wl, rows: int, cols: int, seed: int = 7):
+    import oracle
+    x = W.make_x(wl)
+    r = W.sample_rows(wl.M, rows, seed=seed)
+    xs = x[torch.from_numpy(r)].float().numpy()
+    w = W.make_w(wl, 0)
+    c = W.sample_rows(wl.modules[0], cols, seed=seed + 1)
+    wsub = w[torch.from_numpy(c)].float().numpy()
+    gx = oracle.global_scale(x.float().numpy())
+    gw = oracle.global_scale(w.float().numpy())
+    wc, wsf = oracle.quantize(wsub, gw)                  # offline weight prep, untimed
+    return xs, gx, wc, wsf, gw
+
+
+def time_oracle(wl, seconds: float = 10.0, rows: int = 128, cols: int = 2048):
+    """The oracle (quantize activation rows, float64 dequantize + GEMM) on a
+    bounded sample of the workload, repeated for about `seconds`."""
+    import oracle
+    xs, gx, wc, wsf, gw = oracle_sample(wl, rows, cols)
+    oracle.linear_reference(xs, gx, wc, wsf, gw)          # warm
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.linear_reference(xs, gx, wc, wsf, gw)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    flops = 2.0 * xs.shape[0] * wc.shape[0] * wl.K * reps
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{xs.shape[0]} activation rows x {wc.shape[0]} weight rows x K={wl.K} "
+                      f"(quantize + float64 dequantize/GEMM), {reps} reps in {el:.1f} s; "
+                      f"OpenMP threads {oracle.num_threads()}, numpy BLAS threads as configured"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    import oracle
+    xs, gx, wc, wsf, gw = oracle_sample(wl, 64, 1024)
+    for _ in range(args.warmup):
+        oracle.linear_reference(xs, gx, wc, wsf, gw)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear_reference(xs, gx, wc, wsf, gw)
+    el = time.perf_counter() - t0
+    flops = 2.0 * xs.shape[0] * wc.shape[0] * wl.K * args.steps
+    value = flops / el / 1e12
+    cores = len(os.sched_getaffinity(0))
+    sample = f"{xs.shape[0]} activation rows x {wc.shape[0]} weight rows x K={wl.K} per step"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 quantize, f64 GEMM", "data": "synthetic",
+            "config": {"workload": f"{wl.name} {wl.M}x{wl.N}x{wl.K}", "M": wl.M, "N": wl.N, "K": wl.K},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--headline-only", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        out = run_reference(args)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    out = run_native(args, rank, world, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = time_oracle(W.WORKLOADS[args.workload])
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

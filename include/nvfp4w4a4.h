@@ -1,0 +1,194 @@
+/*
+ * nvfp4w4a4.h -- C ABI of the NVFP4 W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The operation (from the web pages on arXiv 2609.04098, "Why Gated DeltaNet
+ * Survives 4-Bit Quantization: NVFP4 W4A4 for the Recurrent Half of a Hybrid
+ * 27B LLM"):
+ *   - NVFP4 stores 4-bit E2M1 values with one E4M3 scale per 16 consecutive
+ *     elements (the block maximum divided by 6) and one FP32 scale per tensor
+ *     (ta-paperlens page, section "前提1"; arxiv-wiki page, "접근 방법").
+ *   - W4A4: weights and activations are both NVFP4 and the matrix product runs
+ *     on the 4-bit tensor cores (ta-paperlens page, "前提1").
+ *   - Modules that a serving kernel fuses into one GEMM (GDN in_proj_qkv with
+ *     in_proj_z, in_proj_b with in_proj_a) must share one global scale; the
+ *     per-module ratios are folded into the block scales (arxiv-wiki page,
+ *     "접근 방법" and "개발자 관점"; abstract on the shd-paper page).
+ *
+ * Arithmetic (the readings this library implements, bit for bit):
+ *   g       : per-tensor FP32 dequantization scale, g = amax / (6*448)
+ *   g6      = fl32(6 * g)
+ *   s_b     = E4M3_RNE_SATFINITE(fl32(amax_b / g6))     per 16-element block b
+ *   d_b     = fl32(dec(s_b) * g)
+ *   q_i     = E2M1_RNE_SATFINITE(fl32(x_i / d_b))        (+0 codes if dec(s_b)==0 or d_b==0)
+ *   Y[m,n]  = fl32(acc[m,n] * fl32(g_x * g_w)),  acc = sum_k dec(qx)dec(sx)dec(qw)dec(sw)
+ *             accumulated in FP32 by the tensor cores, then rounded to BF16
+ *             (round to nearest even) or kept as FP32.
+ *
+ * Data layouts (all device memory unless stated):
+ *   codes : [rows, K/2] bytes, row stride K/2; element 2j of a row in the low
+ *           nibble of byte j, element 2j+1 in the high nibble.
+ *   sf    : swizzled E4M3 scale bytes of a tensor with R rows:
+ *           nvfp4_sf_bytes(R, K) bytes = pad128(R) * (K/16); the scale of (row r,
+ *           block column c) is at byte
+ *             ((r/128)*(K/64) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4
+ *           (128-row x 4-column atoms of 512 bytes, the layout the sm_100
+ *           block-scaled tensor-core instructions read).  Rows in
+ *           [R, pad128(R)) are padding and hold zero.
+ *   x, y  : row-major with a leading dimension in elements.
+ *
+ * Conventions for every entry point:
+ *   - The caller allocates every buffer (PyTorch in the bundled binding); the
+ *     library never calls cudaMalloc/cudaFree.
+ *   - All work is enqueued on `stream`; nothing synchronizes the host except
+ *     nvfp4_last_device_status().
+ *   - Preconditions: K % 64 == 0, K > 0, rows >= 0; device pointers 16-byte
+ *     aligned; ld_x >= K with ld_x * element size a multiple of 16 bytes;
+ *     ld_y >= N (any value); inputs finite; global scales finite and > 0.
+ *   - Validation failures return a status code before anything is enqueued;
+ *     nothing throws across the ABI.  A CUDA launch error is returned as
+ *     NVFP4_ERR_CUDA.  Kernels bound every wait; a wait that runs out records a
+ *     flag that nvfp4_last_device_status() reports.
+ *   - Calls on one stream are ordered; calls that write the same buffers from
+ *     different streams must be ordered by the caller.
+ */
+#ifndef NVFP4W4A4_H
+#define NVFP4W4A4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nvfp4_stream_t;   /* same object as cudaStream_t; NULL = legacy stream */
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_NULL = 1,        /* a required pointer is NULL */
+    NVFP4_ERR_SHAPE = 2,       /* bad rows/K/M/N/ld or K % 64 != 0 */
+    NVFP4_ERR_ALIGN = 3,       /* a pointer or row stride is not 16-byte aligned */
+    NVFP4_ERR_DTYPE = 4,       /* unknown dtype enum */
+    NVFP4_ERR_UNSUPPORTED = 5, /* valid request this build does not serve */
+    NVFP4_ERR_TIMEOUT = 6,     /* a kernel wait ran out (see nvfp4_last_device_status) */
+    NVFP4_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_WORKSPACE = 8    /* workspace NULL or smaller than the size helper says */
+} nvfp4_status;
+
+typedef enum { NVFP4_IN_BF16 = 0, NVFP4_IN_F32 = 1 } nvfp4_in_dtype;
+typedef enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_F32 = 1 } nvfp4_out_dtype;
+
+/* Bytes of the packed codes of a [rows, K] tensor: rows * K / 2. */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t K);
+
+/* Bytes of the swizzled scale buffer of a [rows, K] tensor: pad128(rows) * K/16. */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
+
+/*
+ * Per-tensor global scale (row a1 of the layer): *gscale_out = amax(|x|)/(6*448),
+ * or 1.0f for an all-zero tensor, where 6 is the largest E2M1 value and 448 the
+ * largest E4M3 value (the pages calibrate this scale offline per module,
+ * arxiv-wiki page "접근 방법"; this call computes it from the tensor itself).
+ *   x          : [rows, K] of dtype dt, row stride ld_x elements (device).
+ *   gscale_out : 1 float (device); also used as the reduction accumulator, so
+ *                it must not alias x.
+ */
+nvfp4_status nvfp4_amax_gscale(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K,
+                               int64_t ld_x, float *gscale_out, nvfp4_stream_t stream);
+
+/*
+ * Quantize a [rows, K] tensor to NVFP4 (rows a2, a3 and a5 of the layer;
+ * ta-paperlens page "前提1").
+ *   x         : [rows, K] bf16 or fp32 (dt), row stride ld_x elements (device).
+ *   gscale    : 1 float, the tensor's global scale g (device).
+ *   codes     : [rows, K/2] bytes for THIS call's rows (device, written).
+ *   sf        : base of the swizzled scale buffer of a tensor with
+ *               sf_rows_total rows (device, nvfp4_sf_bytes(sf_rows_total, K)
+ *               bytes); this call writes the scales of rows
+ *               [sf_row0, sf_row0 + rows).  When sf_row0 + rows == sf_rows_total
+ *               it also zeroes the padding rows [sf_rows_total, pad128(sf_rows_total)).
+ *   sf_row0, sf_rows_total : place the tensor inside a fused (concatenated
+ *               along rows) weight, so each module is quantized with its own g
+ *               and then harmonized (nvfp4_harmonize_group).
+ */
+nvfp4_status nvfp4_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K,
+                            int64_t ld_x, const float *gscale, uint8_t *codes, uint8_t *sf,
+                            int64_t sf_row0, int64_t sf_rows_total, nvfp4_stream_t stream);
+
+/*
+ * Fused-group global-scale repair (row a6; arxiv-wiki page "접근 방법", last
+ * bullet, and "개발자 관점": per-module-calibrated checkpoints served by a
+ * kernel that fuses the modules into one GEMM need one shared global scale,
+ * with the ratios folded into the block scales).
+ *   sf            : fused swizzled scale buffer, rows_total rows (device, in place).
+ *   row_offsets   : n_modules + 1 HOST integers, 0 = row_offsets[0] < ... <
+ *                   row_offsets[n_modules] = rows_total; module m owns rows
+ *                   [row_offsets[m], row_offsets[m+1]).
+ *   gscales       : n_modules floats, each module's own global scale (device).
+ *   shared_gscale_out : 1 float (device): g* = max_m gscales[m].  Must not
+ *                   alias gscales.
+ * Every scale byte s of module m becomes E4M3_RNE_SATFINITE(fl32(dec(s) *
+ * fl32(g_m / g*))); the codes are unchanged.  1 <= n_modules <= 16.
+ */
+nvfp4_status nvfp4_harmonize_group(uint8_t *sf, int64_t rows_total, int64_t K, int n_modules,
+                                   const int64_t *row_offsets, const float *gscales,
+                                   float *shared_gscale_out, nvfp4_stream_t stream);
+
+/*
+ * Block-scaled W4A4 GEMM on pre-quantized operands (rows a7, a8):
+ *   y[m, n] = fl32(acc * fl32(a_gscale * b_gscale)),
+ *   acc[m, n] = sum_k dec(a)[m,k] * dec(b)[n,k]  (tcgen05 kind::mxf4nvf4, FP32 in TMEM)
+ *   a_codes/a_sf : activation, M rows (device); a_sf has nvfp4_sf_bytes(M, K) bytes.
+ *   b_codes/b_sf : weight, N rows (device); b_sf has nvfp4_sf_bytes(N, K) bytes.
+ *   a_gscale, b_gscale : 1 float each (device).
+ *   y            : [M, N] bf16 or fp32 (y_dt), row stride ld_y elements (device).
+ *   workspace    : device scratch of at least nvfp4_gemm_workspace_bytes(M, N, K)
+ *                  bytes (may be NULL when that is 0).
+ */
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
+                        const uint8_t *b_codes, const uint8_t *b_sf, const float *b_gscale,
+                        void *y, nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N,
+                        int64_t K, void *workspace, size_t workspace_bytes,
+                        nvfp4_stream_t stream);
+
+/*
+ * The W4A4 linear layer (all rows a2-a9): quantize the activation x on the
+ * fly with its global scale, then the block-scaled GEMM against pre-quantized
+ * NVFP4 weights (ta-paperlens page "前提1": both operands 4-bit, product on
+ * 4-bit tensor cores).
+ *   x        : [M, K] bf16 or fp32 (x_dt), row stride ld_x elements (device).
+ *   x_gscale : 1 float (device).
+ *   w_codes, w_sf, w_gscale : the weight as written by nvfp4_quantize (and,
+ *              for a fused group, nvfp4_harmonize_group's shared scale).
+ *   y        : [M, N] (y_dt), row stride ld_y (device).
+ *   workspace: device scratch, >= w4a4_gemm_workspace_bytes(M, N, K) bytes;
+ *              holds the quantized activation and any split-K partial sums.
+ */
+size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                       const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale,
+                       void *y, nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N,
+                       int64_t K, void *workspace, size_t workspace_bytes,
+                       nvfp4_stream_t stream);
+
+/*
+ * Synchronizes the device, then reports and clears the library's device error
+ * word: *flags receives the OR of the flags kernels recorded since the last
+ * call (bit 0: a producer wait ran out, bit 1: an MMA wait ran out, bit 2: an
+ * epilogue wait ran out, bit 3: a TMEM allocation wait ran out).  Returns
+ * NVFP4_ERR_TIMEOUT if any flag was set, NVFP4_ERR_CUDA on a CUDA error.
+ */
+nvfp4_status nvfp4_last_device_status(int *flags);
+
+/* Static string for a status code. */
+const char *nvfp4_status_string(nvfp4_status status);
+
+/* Number of kernel launches this library has enqueued in this process. */
+uint64_t nvfp4_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4W4A4_H */

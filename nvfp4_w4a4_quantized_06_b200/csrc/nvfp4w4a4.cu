@@ -1,0 +1,427 @@
+// nvfp4w4a4.cu -- the C ABI of the NVFP4 W4A4 linear layer (declared in
+// include/nvfp4w4a4.h): argument validation, TMA tensor-map encoding, shape
+// dispatch and kernel launches.  No entry point allocates device memory; the
+// only library state is a per-device error word and a few cached attributes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "nvfp4w4a4.h"
+#include "ptx.cuh"
+#include "quantize.cuh"
+#include "gemm.cuh"
+
+using namespace nvfp4;
+
+__device__ unsigned g_nvfp4_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  unsigned *err = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t pad128(int64_t r) { return (r + 127) / 128 * 128; }
+inline size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int BN>
+cudaError_t set_gemm_attrs() {
+  const int b = GemmCfg<BN>::SMEM_BYTES;
+  cudaError_t e = set_smem(nvfp4_gemm_kernel<BN, OUT_BF16>, b);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_kernel<BN, OUT_F32>, b);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_kernel<BN, OUT_PARTIAL>, b);
+  return e;
+}
+
+// Per-device one-time setup with the device current: SM count, the address of
+// the error word, the kernels' shared-memory limits, the tensor-map encoder.
+nvfp4_status device_state(DeviceState **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState &d = g_dev[dev];
+  if (!d.ready) {
+    if (!g_encode) {
+      void *fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return NVFP4_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    int sms = 0, major = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (major != 10) return NVFP4_ERR_UNSUPPORTED;
+    void *errp = nullptr;
+    if (cudaGetSymbolAddress(&errp, g_nvfp4_device_error) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (set_gemm_attrs<256>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
+        set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<32>() != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    d.sms = sms;
+    d.err = static_cast<unsigned *>(errp);
+    d.ready = true;
+  }
+  *out = &d;
+  return NVFP4_OK;
+}
+
+nvfp4_status launched() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+bool make_codes_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// GEMM plan: which operand drives the 128-row MMA dimension, the tile width,
+// split-K and the grid.
+struct Plan {
+  bool swap;       // A operand = weight (rows N), B operand = activation (rows M)
+  int bn;
+  int tiles_a, tiles_b, splits, kstages;
+  int grid;
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int sms) {
+  Plan pl{};
+  pl.kstages = (int)((K / 64 + 3) / 4);
+  if (M <= 64) {
+    // decode-shaped: the weight streams through the 128-row MMA dimension and
+    // the few activation rows are the MMA's N; split K so that every SM
+    // (two CTAs each) streams a share of the weight
+    pl.swap = true;
+    pl.bn = M <= 32 ? 32 : 64;
+    pl.tiles_a = (int)((N + 127) / 128);
+    pl.tiles_b = 1;
+    int s = (2 * sms) / pl.tiles_a;
+    pl.splits = s < 1 ? 1 : (s > pl.kstages ? pl.kstages : s);
+  } else {
+    pl.swap = false;
+    pl.bn = N <= 128 ? 128 : 256;
+    pl.tiles_a = (int)((M + 127) / 128);
+    pl.tiles_b = (int)((N + pl.bn - 1) / pl.bn);
+    const int units = pl.tiles_a * pl.tiles_b;
+    int s = units < sms ? sms / units : 1;
+    if (s > pl.kstages / 2) s = pl.kstages / 2;
+    pl.splits = s < 1 ? 1 : s;
+  }
+  const int units = pl.tiles_a * pl.tiles_b * pl.splits;
+  const int per_sm = pl.bn <= 64 ? 2 : 1;
+  pl.grid = units < per_sm * sms ? units : per_sm * sms;
+  return pl;
+}
+
+size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, int sms) {
+  const Plan pl = make_plan(M, N, K, sms);
+  return pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
+}
+
+int current_sms() {
+  DeviceState *d = nullptr;
+  if (device_state(&d) != NVFP4_OK) return 148;
+  return d->sms;
+}
+
+template <int BN>
+nvfp4_status launch_gemm_bn(const CUtensorMap &ma, const CUtensorMap &mb, const GemmParams &p, int mode,
+                            int grid, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  if (mode == OUT_BF16)
+    nvfp4_gemm_kernel<BN, OUT_BF16><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mb, p);
+  else if (mode == OUT_F32)
+    nvfp4_gemm_kernel<BN, OUT_F32><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mb, p);
+  else
+    nvfp4_gemm_kernel<BN, OUT_PARTIAL><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mb, p);
+  return launched();
+}
+
+nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
+                       const uint8_t *b_codes, const uint8_t *b_sf, const float *b_gscale, void *y,
+                       nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K, void *ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  const Plan pl = make_plan(M, N, K, dev->sms);
+  const size_t need = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
+  if (need > 0 && (ws == nullptr || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(ws)) return NVFP4_ERR_ALIGN;
+
+  GemmParams p{};
+  const uint8_t *op_a = pl.swap ? b_codes : a_codes;   // A = 128-row MMA operand
+  const uint8_t *op_b = pl.swap ? a_codes : b_codes;
+  p.sfa = pl.swap ? b_sf : a_sf;
+  p.sfb = pl.swap ? a_sf : b_sf;
+  p.ga = a_gscale;
+  p.gb = b_gscale;
+  p.rows_a = (int)(pl.swap ? N : M);
+  p.rows_b = (int)(pl.swap ? M : N);
+  p.K = (int)K;
+  p.kblocks = (int)(K / 64);
+  p.kstages = pl.kstages;
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.splits = pl.splits;
+  p.group = 16;
+  p.err = dev->err;
+  int mode;
+  if (pl.splits > 1) {
+    mode = OUT_PARTIAL;
+    p.out = ws;
+    p.part_stride = M * N;
+    p.out_si = pl.swap ? 1 : N;      // partials in output coordinates [m][n]
+    p.out_sj = pl.swap ? N : 1;
+  } else {
+    mode = y_dt == NVFP4_OUT_BF16 ? OUT_BF16 : OUT_F32;
+    p.out = y;
+    p.out_si = pl.swap ? 1 : ld_y;
+    p.out_sj = pl.swap ? ld_y : 1;
+  }
+  CUtensorMap ma, mb;
+  if (!make_codes_map(&ma, op_a, p.rows_a, K, 128) || !make_codes_map(&mb, op_b, p.rows_b, K, pl.bn))
+    return NVFP4_ERR_CUDA;
+  switch (pl.bn) {
+    case 256: st = launch_gemm_bn<256>(ma, mb, p, mode, pl.grid, stream); break;
+    case 128: st = launch_gemm_bn<128>(ma, mb, p, mode, pl.grid, stream); break;
+    case 64: st = launch_gemm_bn<64>(ma, mb, p, mode, pl.grid, stream); break;
+    default: st = launch_gemm_bn<32>(ma, mb, p, mode, pl.grid, stream); break;
+  }
+  if (st != NVFP4_OK || pl.splits == 1) return st;
+  const int64_t MN = M * N;
+  int grid = (int)((MN + 255) / 256);
+  if (grid > 8 * dev->sms) grid = 8 * dev->sms;
+  if (y_dt == NVFP4_OUT_BF16)
+    splitk_reduce_kernel<OUT_BF16><<<grid, 256, 0, stream>>>(static_cast<const float *>(ws), pl.splits, MN,
+                                                             (int)N, a_gscale, b_gscale, y, ld_y);
+  else
+    splitk_reduce_kernel<OUT_F32><<<grid, 256, 0, stream>>>(static_cast<const float *>(ws), pl.splits, MN,
+                                                            (int)N, a_gscale, b_gscale, y, ld_y);
+  return launched();
+}
+
+nvfp4_status check_gemm_args(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
+                             const uint8_t *b_codes, const uint8_t *b_sf, const float *b_gscale,
+                             const void *y, int y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > (1 << 30))
+    return NVFP4_ERR_SHAPE;
+  if (y_dt != NVFP4_OUT_BF16 && y_dt != NVFP4_OUT_F32) return NVFP4_ERR_DTYPE;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!a_codes || !a_sf || !a_gscale || !b_codes || !b_sf || !b_gscale || !y) return NVFP4_ERR_NULL;
+  if (ld_y < N) return NVFP4_ERR_SHAPE;
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_sf) || !aligned16(b_sf) || !aligned16(y))
+    return NVFP4_ERR_ALIGN;
+  return NVFP4_OK;
+}
+
+template <typename T>
+void launch_quantize(const QuantizeParams &p, int sms, cudaStream_t s) {
+  constexpr int U = 4;
+  const int64_t nseg = (p.K + 255) / 256;
+  const int64_t units = p.rows * nseg;
+  int64_t blocks = ((units + U - 1) / U + 7) / 8;
+  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  if (blocks < 1) blocks = 1;
+  quantize_kernel<T, U><<<(unsigned)blocks, 256, 0, s>>>(p);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_codes_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0) return 0;
+  return (size_t)rows * (size_t)(K / 2);
+}
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0) return 0;
+  return (size_t)pad128(rows) * (size_t)((K / 16 + 3) / 4 * 4);
+}
+
+nvfp4_status nvfp4_amax_gscale(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                               float *gscale_out, nvfp4_stream_t stream) {
+  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K) return NVFP4_ERR_SHAPE;
+  if (!gscale_out || (rows > 0 && !x)) return NVFP4_ERR_NULL;
+  const int esz = dt == NVFP4_IN_BF16 ? 2 : 4;
+  if ((rows > 0 && !aligned16(x)) || (ld_x * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(gscale_out) & 3))
+    return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(gscale_out, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (rows > 0) {
+    int64_t n = rows * (K / 8);
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
+    unsigned *acc = reinterpret_cast<unsigned *>(gscale_out);
+    if (dt == NVFP4_IN_BF16)
+      amax_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), rows, K,
+                                                                  ld_x, acc);
+    else
+      amax_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float *>(x), rows, K, ld_x, acc);
+    if ((st = launched()) != NVFP4_OK) return st;
+  }
+  gscale_finalize_kernel<<<1, 1, 0, s>>>(reinterpret_cast<unsigned *>(gscale_out));
+  return launched();
+}
+
+nvfp4_status nvfp4_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                            const float *gscale, uint8_t *codes, uint8_t *sf, int64_t sf_row0,
+                            int64_t sf_rows_total, nvfp4_stream_t stream) {
+  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || sf_row0 < 0 || sf_rows_total < sf_row0 + rows)
+    return NVFP4_ERR_SHAPE;
+  const bool owns_pad = sf_row0 + rows == sf_rows_total;
+  const int64_t pad_rows = owns_pad ? pad128(sf_rows_total) - sf_rows_total : 0;
+  if (rows == 0 && pad_rows == 0) return NVFP4_OK;
+  if (!sf || !gscale || (rows > 0 && (!x || !codes))) return NVFP4_ERR_NULL;
+  const int esz = dt == NVFP4_IN_BF16 ? 2 : 4;
+  if ((rows > 0 && (!aligned16(x) || !aligned16(codes))) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  QuantizeParams p{x, rows, K, ld_x, gscale, codes, sf, sf_row0, pad_rows};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dt == NVFP4_IN_BF16) launch_quantize<__nv_bfloat16>(p, dev->sms, s);
+  else launch_quantize<float>(p, dev->sms, s);
+  return launched();
+}
+
+nvfp4_status nvfp4_harmonize_group(uint8_t *sf, int64_t rows_total, int64_t K, int n_modules,
+                                   const int64_t *row_offsets, const float *gscales, float *shared_gscale_out,
+                                   nvfp4_stream_t stream) {
+  if (!sf || !row_offsets || !gscales || !shared_gscale_out) return NVFP4_ERR_NULL;
+  if (n_modules < 1 || n_modules > kMaxModules || rows_total <= 0 || K <= 0 || K % 64 != 0)
+    return NVFP4_ERR_SHAPE;
+  if (row_offsets[0] != 0 || row_offsets[n_modules] != rows_total) return NVFP4_ERR_SHAPE;
+  for (int m = 0; m < n_modules; ++m)
+    if (row_offsets[m + 1] <= row_offsets[m]) return NVFP4_ERR_SHAPE;
+  if (!aligned16(sf)) return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  HarmonizeParams p{};
+  p.sf = sf;
+  p.rows_total = rows_total;
+  p.K = K;
+  p.n = n_modules;
+  for (int m = 0; m <= n_modules; ++m) p.offs[m] = row_offsets[m];
+  p.gs = gscales;
+  p.gstar_out = shared_gscale_out;
+  const int64_t total = rows_total * (K / 64);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
+  if (blocks < 1) blocks = 1;
+  harmonize_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return launched();
+}
+
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
+  return gemm_partial_bytes(M, N, K, current_sms());
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
+                        const uint8_t *b_codes, const uint8_t *b_sf, const float *b_gscale, void *y,
+                        nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K, void *workspace,
+                        size_t workspace_bytes, nvfp4_stream_t stream) {
+  nvfp4_status st = check_gemm_args(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, y, y_dt, ld_y, M, N, K);
+  if (st != NVFP4_OK || M == 0 || N == 0) return st;
+  return gemm_impl(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, y, y_dt, ld_y, M, N, K, workspace,
+                   workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
+  return align256(nvfp4_codes_bytes(M, K)) + align256(nvfp4_sf_bytes(M, K)) +
+         gemm_partial_bytes(M, N, K, current_sms());
+}
+
+nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                       const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
+                       nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K, void *workspace,
+                       size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (x_dt != NVFP4_IN_BF16 && x_dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ld_x < K) return NVFP4_ERR_SHAPE;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!x || !x_gscale) return NVFP4_ERR_NULL;
+  const int esz = x_dt == NVFP4_IN_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+  if (!workspace) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return NVFP4_ERR_ALIGN;
+  const size_t codes_b = align256(nvfp4_codes_bytes(M, K));
+  const size_t sf_b = align256(nvfp4_sf_bytes(M, K));
+  if (workspace_bytes < codes_b + sf_b) return NVFP4_ERR_WORKSPACE;
+  uint8_t *a_codes = static_cast<uint8_t *>(workspace);
+  uint8_t *a_sf = a_codes + codes_b;
+  nvfp4_status st = check_gemm_args(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K);
+  if (st != NVFP4_OK) return st;
+  DeviceState *dev = nullptr;
+  if ((st = device_state(&dev)) != NVFP4_OK) return st;
+  if (workspace_bytes < codes_b + sf_b + gemm_partial_bytes(M, N, K, dev->sms)) return NVFP4_ERR_WORKSPACE;
+  st = nvfp4_quantize(x, x_dt, M, K, ld_x, x_gscale, a_codes, a_sf, 0, M, stream);
+  if (st != NVFP4_OK) return st;
+  return gemm_impl(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K,
+                   a_sf + sf_b, workspace_bytes - codes_b - sf_b, reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_last_device_status(int *flags) {
+  if (!flags) return NVFP4_ERR_NULL;
+  *flags = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return NVFP4_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_nvfp4_device_error, sizeof(v)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_nvfp4_device_error, &zero, sizeof(zero)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  *flags = (int)v;
+  return v ? NVFP4_ERR_TIMEOUT : NVFP4_OK;
+}
+
+const char *nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_NULL: return "null pointer";
+    case NVFP4_ERR_SHAPE: return "bad shape";
+    case NVFP4_ERR_ALIGN: return "misaligned pointer or stride";
+    case NVFP4_ERR_DTYPE: return "unknown dtype";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device)";
+    case NVFP4_ERR_TIMEOUT: return "a kernel wait ran out";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,221 @@
+// quantize.cuh -- NVFP4 encoder kernels for sm_100a: per-tensor global scale,
+// activation/weight quantize (E2M1 codes + swizzled E4M3 block scales) and
+// fused-group global-scale harmonization.
+//
+// Format (web pages on arXiv 2609.04098; ta-paperlens page, section "前提1";
+// arxiv-wiki page, "접근 방법"): 4-bit E2M1 values, one E4M3 scale per 16
+// consecutive elements equal to the block maximum / 6, and one FP32 scale per
+// tensor.  Arithmetic per block (each step one IEEE fp32 operation):
+//   g6 = 6*g;  s = E4M3(amax/g6);  d = dec(s)*g;  q_i = E2M1(x_i/d)
+// with round-to-nearest-even and saturation at 448 / 6; a block whose scale
+// or d is zero gets +0 codes.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+// byte offset of the scale of (row r, block column c) in the swizzled buffer
+// (128-row x 4-column atoms of 512 bytes; K % 64 == 0 so K/64 atoms per row block)
+__device__ __forceinline__ int64_t sf_index(int64_t r, int64_t c, int64_t K) {
+  return ((r >> 7) * (K >> 6) + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+template <typename T>
+struct Vec8;  // eight consecutive input elements as fp32
+
+template <>
+struct Vec8<__nv_bfloat16> {
+  uint4 raw;
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+    raw = __ldg(reinterpret_cast<const uint4 *>(p));
+  }
+  __device__ __forceinline__ void to_f32(float (&v)[8]) const {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+
+template <>
+struct Vec8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *p) {
+    a = __ldg(reinterpret_cast<const float4 *>(p));
+    b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  }
+  __device__ __forceinline__ void to_f32(float (&v)[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+// Encode eight values of one half-block given the block's amax; returns the
+// packed code word and (through *s_out) the E4M3 scale byte.
+__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float amax, float g, float g6,
+                                            uint32_t *s_out) {
+  const float t = __fdiv_rn(amax, g6);
+  const uint32_t s = f32_to_e4m3(t);
+  const float decs = e4m3_to_f32(s);
+  const float d = __fmul_rn(decs, g);
+  *s_out = s;
+  if (decs == 0.0f || d == 0.0f) return 0u;
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(v[i], d);
+  return f32x8_to_e2m1(y);
+}
+
+struct QuantizeParams {
+  const void *x;
+  int64_t rows, K, ld_x;
+  const float *gscale;
+  uint8_t *codes;
+  uint8_t *sf;
+  int64_t sf_row0;
+  int64_t pad_rows;  // padding rows (zeroed) after this call's rows, or 0
+};
+
+// One warp handles a 256-element segment of one row per unit: lane l owns
+// elements [8l, 8l+8), lanes 2i and 2i+1 form 16-element block i and exchange
+// their half-maxima with one shuffle.  Loads are 16-byte vectors (a warp reads
+// 512 contiguous bytes of bf16), code words are 4-byte stores (128 contiguous
+// bytes per warp).  UNROLL units are loaded before any is encoded.
+template <typename T, int UNROLL>
+__global__ void __launch_bounds__(256) quantize_kernel(QuantizeParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t nseg = (p.K + 255) >> 8;
+  const int64_t units = p.rows * nseg;
+  const int64_t ncols = p.K >> 4;
+  const float g = __ldg(p.gscale);
+  const float g6 = __fmul_rn(6.0f, g);
+  const T *x = static_cast<const T *>(p.x);
+
+  for (int64_t u0 = warp * UNROLL; u0 < units; u0 += nwarps * UNROLL) {
+    Vec8<T> in[UNROLL];
+#pragma unroll
+    for (int j = 0; j < UNROLL; ++j) {
+      const int64_t u = u0 + j;
+      const int64_t row = u / nseg, col = (u - row * nseg) * 256 + lane * 8;
+      if (u < units && col < p.K) in[j].load(x + row * p.ld_x + col);
+    }
+#pragma unroll
+    for (int j = 0; j < UNROLL; ++j) {
+      const int64_t u = u0 + j;
+      const int64_t row = u / nseg, col = (u - row * nseg) * 256 + lane * 8;
+      const bool active = u < units && col < p.K;
+      float v[8];
+      in[j].to_f32(v);
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      if (!active) amax = 0.0f;
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      if (active) {
+        uint32_t s;
+        const uint32_t word = encode8(v, amax, g, g6, &s);
+        *reinterpret_cast<uint32_t *>(p.codes + row * (p.K >> 1) + (col >> 1)) = word;
+        if ((lane & 1) == 0) p.sf[sf_index(p.sf_row0 + row, col >> 4, p.K)] = static_cast<uint8_t>(s);
+      }
+    }
+  }
+  // zero the scale bytes of the padding rows this call owns
+  const int64_t pad_bytes = p.pad_rows * ncols;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = tid; i < pad_bytes; i += nthreads) {
+    const int64_t r = p.sf_row0 + p.rows + i / ncols, c = i % ncols;
+    p.sf[sf_index(r, c, p.K)] = 0;
+  }
+}
+
+// ------------------------------------------------------------- global scale
+template <typename T>
+__global__ void __launch_bounds__(256) amax_kernel(const T *x, int64_t rows, int64_t K, int64_t ld,
+                                                   unsigned *amax_bits) {
+  const int64_t chunks_per_row = K >> 3;
+  const int64_t n = rows * chunks_per_row;
+  float m = 0.0f;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / chunks_per_row, c = (i - r * chunks_per_row) * 8;
+    Vec8<T> v8;
+    v8.load(x + r * ld + c);
+    float v[8];
+    v8.to_f32(v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+    // non-negative floats order like their bit patterns
+    atomicMax(amax_bits, __float_as_uint(m));
+  }
+}
+
+// g = amax / (6*448), or 1 for an all-zero tensor; rewrites the word in place
+__global__ void gscale_finalize_kernel(unsigned *amax_bits) {
+  const float a = __uint_as_float(*amax_bits);
+  const float g = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
+  *reinterpret_cast<float *>(amax_bits) = g;
+}
+
+// ---------------------------------------------------------------- harmonize
+constexpr int kMaxModules = 16;
+
+struct HarmonizeParams {
+  uint8_t *sf;
+  int64_t rows_total, K;
+  int n;
+  int64_t offs[kMaxModules + 1];
+  const float *gs;
+  float *gstar_out;
+};
+
+// One thread per (row, 4 block columns) = one 32-bit word of the swizzled
+// buffer.  g* = max_m g_m; each scale byte of module m becomes
+// E4M3(dec(s) * (g_m / g*)).
+__global__ void __launch_bounds__(256) harmonize_kernel(HarmonizeParams p) {
+  __shared__ float ratio[kMaxModules];
+  __shared__ float gstar_s;
+  if (threadIdx.x == 0) {
+    float gstar = __ldg(p.gs);
+    for (int m = 1; m < p.n; ++m) gstar = fmaxf(gstar, __ldg(p.gs + m));
+    gstar_s = gstar;
+    for (int m = 0; m < p.n; ++m) ratio[m] = __fdiv_rn(__ldg(p.gs + m), gstar);
+  }
+  __syncthreads();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.gstar_out = gstar_s;
+  const int64_t words_per_row = p.K >> 6;
+  const int64_t total = p.rows_total * words_per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / words_per_row, cw = i - r * words_per_row;
+    int m = 0;
+    while (m + 1 < p.n && r >= p.offs[m + 1]) ++m;
+    const float rt = ratio[m];
+    uint32_t *w = reinterpret_cast<uint32_t *>(p.sf + sf_index(r, cw * 4, p.K));
+    const uint32_t in = *w;
+    uint32_t out = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float v = __fmul_rn(e4m3_to_f32((in >> (8 * b)) & 0xFFu), rt);
+      out |= f32_to_e4m3(v) << (8 * b);
+    }
+    *w = out;
+  }
+}
+
+}  // namespace nvfp4

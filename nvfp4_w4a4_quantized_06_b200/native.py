@@ -1,0 +1,189 @@
+"""ctypes binding of libnvfp4w4a4.so (the C ABI in include/nvfp4w4a4.h).
+
+Argument marshalling only: torch allocates the outputs and supplies the
+current CUDA stream; every step of the layer runs in the library's kernels.
+There is no fallback: if the library is missing or the call fails, this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4w4a4.so")
+
+IN_BF16, IN_F32 = 0, 1
+OUT_BF16, OUT_F32 = 0, 1
+STATUS = {0: "ok", 1: "null pointer", 2: "bad shape", 3: "misaligned", 4: "bad dtype",
+          5: "unsupported", 6: "timeout", 7: "CUDA error", 8: "workspace"}
+
+_lib = None
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m nvfp4_w4a4_quantized_06_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.nvfp4_codes_bytes.argtypes, L.nvfp4_codes_bytes.restype = [i64, i64], sz
+        L.nvfp4_sf_bytes.argtypes, L.nvfp4_sf_bytes.restype = [i64, i64], sz
+        L.nvfp4_amax_gscale.argtypes = [vp, i32, i64, i64, i64, vp, vp]
+        L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i64, i64, vp]
+        L.nvfp4_harmonize_group.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
+        L.nvfp4_gemm_workspace_bytes.argtypes, L.nvfp4_gemm_workspace_bytes.restype = [i64, i64, i64], sz
+        L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, sz, vp]
+        L.w4a4_gemm_workspace_bytes.argtypes, L.w4a4_gemm_workspace_bytes.restype = [i64, i64, i64], sz
+        L.w4a4_gemm.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, sz, vp]
+        L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
+        L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
+        for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
+                  "w4a4_gemm", "nvfp4_last_device_status"):
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise Nvfp4Error(fn, status)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _in_dtype(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return IN_BF16
+    if x.dtype == torch.float32:
+        return IN_F32
+    raise TypeError(f"unsupported input dtype {x.dtype}")
+
+
+def _out_dtype(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return OUT_BF16
+    if dt == torch.float32:
+        return OUT_F32
+    raise TypeError(f"unsupported output dtype {dt}")
+
+
+def _require_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live on the GPU")
+
+
+def codes_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_codes_bytes(rows, K))
+
+
+def sf_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_sf_bytes(rows, K))
+
+
+def amax_gscale(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Per-tensor global scale amax/(6*448) as a 1-element fp32 device tensor."""
+    _require_cuda(x)
+    rows, K = x.shape
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    _check("nvfp4_amax_gscale", lib().nvfp4_amax_gscale(_ptr(x), _in_dtype(x), rows, K, x.stride(0),
+                                                         _ptr(out), _stream()))
+    return out
+
+
+def quantize(x: torch.Tensor, gscale: torch.Tensor, codes: torch.Tensor | None = None,
+             sf: torch.Tensor | None = None, sf_row0: int = 0, sf_rows_total: int | None = None):
+    """NVFP4-quantize x [rows, K]; returns (codes [rows, K/2] uint8, sf uint8 swizzled)."""
+    _require_cuda(x, gscale)
+    rows, K = x.shape
+    total = rows if sf_rows_total is None else sf_rows_total
+    if codes is None:
+        codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(sf_bytes(total, K), dtype=torch.uint8, device=x.device)
+    _check("nvfp4_quantize", lib().nvfp4_quantize(_ptr(x), _in_dtype(x), rows, K, x.stride(0), _ptr(gscale),
+                                                   _ptr(codes), _ptr(sf), sf_row0, total, _stream()))
+    return codes, sf
+
+
+def harmonize(sf: torch.Tensor, rows_total: int, K: int, row_offsets, gscales: torch.Tensor,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """Rewrite a fused group's scales to one shared global scale; returns g*."""
+    _require_cuda(sf, gscales)
+    offs = (ctypes.c_int64 * len(row_offsets))(*[int(o) for o in row_offsets])
+    out = torch.empty(1, dtype=torch.float32, device=sf.device) if out is None else out
+    _check("nvfp4_harmonize_group", lib().nvfp4_harmonize_group(
+        _ptr(sf), rows_total, K, len(row_offsets) - 1, ctypes.cast(offs, ctypes.c_void_p),
+        _ptr(gscales), _ptr(out), _stream()))
+    return out
+
+
+def gemm(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, out_dtype=torch.bfloat16,
+         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Y[M, N] = (ga*gb) * dec(A) @ dec(B)^T on pre-quantized NVFP4 operands."""
+    _require_cuda(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a_codes.device)
+    need = int(lib().nvfp4_gemm_workspace_bytes(M, N, K))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=a_codes.device)
+    _check("nvfp4_gemm", lib().nvfp4_gemm(
+        _ptr(a_codes), _ptr(a_sf), _ptr(a_gscale), _ptr(b_codes), _ptr(b_sf), _ptr(b_gscale),
+        _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream()))
+    return out
+
+
+def linear_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().w4a4_gemm_workspace_bytes(M, N, K))
+
+
+def linear(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
+           w_gscale: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The W4A4 linear: on-the-fly NVFP4 quantize of x, then the block-scaled GEMM."""
+    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=x.device)
+    _check("w4a4_gemm", lib().w4a4_gemm(
+        _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
+        _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _ptr(workspace), workspace.numel(),
+        _stream()))
+    return out
+
+
+def last_device_status() -> int:
+    """Synchronize, then return and clear the device error flags (0 = clean)."""
+    flags = ctypes.c_int(0)
+    st = lib().nvfp4_last_device_status(ctypes.byref(flags))
+    if st not in (0, 6):
+        raise Nvfp4Error("nvfp4_last_device_status", st)
+    return flags.value
+
+
+def launch_count() -> int:
+    return int(lib().nvfp4_launch_count())

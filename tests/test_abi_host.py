@@ -1,0 +1,94 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/nvfp4w4a4.h declares, and rejects bad arguments with
+the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_w4a4_quantized_06_b200 import build, native
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "nvfp4w4a4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return native.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][A-Za-z0-9_ \*]*?\b((?:nvfp4|w4a4)_[a-z0-9_]+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_size_helpers(L):
+    assert L.nvfp4_codes_bytes(64, 256) == 64 * 128
+    assert L.nvfp4_sf_bytes(64, 256) == 128 * 16
+    assert L.nvfp4_sf_bytes(129, 5120) == 256 * 320
+    assert L.nvfp4_codes_bytes(-1, 64) == 0
+
+
+def test_status_strings(L):
+    for s in range(9):
+        assert L.nvfp4_status_string(s)
+
+
+FAKE = 1 << 20   # a 16-byte-aligned non-null stand-in; validation fails before any use
+
+
+def test_quantize_validation(L):
+    q = L.nvfp4_quantize
+    assert q(FAKE, 7, 4, 64, 64, FAKE, FAKE, FAKE, 0, 4, None) == 4            # dtype
+    assert q(FAKE, 0, 4, 100, 100, FAKE, FAKE, FAKE, 0, 4, None) == 2          # K % 64
+    assert q(FAKE, 0, 4, 64, 32, FAKE, FAKE, FAKE, 0, 4, None) == 2           # ld < K
+    assert q(FAKE, 0, 4, 64, 64, FAKE, FAKE, FAKE, 2, 4, None) == 2           # rows past the fused total
+    assert q(None, 0, 4, 64, 64, FAKE, FAKE, FAKE, 0, 4, None) == 1           # null x
+    assert q(FAKE + 2, 0, 4, 64, 64, FAKE, FAKE, FAKE, 0, 4, None) == 3       # misaligned x
+    assert q(FAKE, 0, 4, 64, 68, FAKE, FAKE, FAKE, 0, 4, None) == 3           # row stride not 16 B
+
+
+def test_gemm_validation(L):
+    g = L.nvfp4_gemm
+    args = [FAKE] * 7
+    assert g(*args, 0, 64, 8, 64, 100, None, 0, None) == 2                    # K % 64
+    assert g(*args, 5, 64, 8, 64, 128, None, 0, None) == 4                    # out dtype
+    assert g(*args, 0, 32, 8, 64, 128, None, 0, None) == 2                    # ld_y < N
+    assert g(None, *args[1:], 0, 64, 8, 64, 128, None, 0, None) == 1          # null
+    assert g(*args[:6], FAKE + 4, 0, 64, 8, 64, 128, None, 0, None) == 3      # misaligned y
+
+
+def test_linear_validation(L):
+    w = L.w4a4_gemm
+    assert w(FAKE, 0, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 8, 64, 256, None, 0, None) == 8   # no workspace
+    assert w(FAKE, 0, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 8, 64, 256, FAKE, 16, None) == 8  # too small
+    assert w(FAKE, 3, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 8, 64, 256, FAKE, 0, None) == 4
+    assert w(FAKE, 0, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 8, 64, 256, FAKE, 0, None) == 2
+
+
+def test_harmonize_validation(L):
+    h = L.nvfp4_harmonize_group
+    offs = (ctypes.c_int64 * 3)(0, 48, 96)
+    bad = (ctypes.c_int64 * 3)(0, 48, 90)
+    po = ctypes.cast(offs, ctypes.c_void_p)
+    assert h(FAKE, 96, 256, 2, ctypes.cast(bad, ctypes.c_void_p), FAKE, FAKE, None) == 2
+    assert h(FAKE, 96, 256, 0, po, FAKE, FAKE, None) == 2
+    assert h(FAKE, 96, 256, 17, po, FAKE, FAKE, None) == 2
+    assert h(None, 96, 256, 2, po, FAKE, FAKE, None) == 1
+    assert h(FAKE, 96, 100, 2, po, FAKE, FAKE, None) == 2
+
+
+def test_empty_inputs_are_no_ops(L):
+    # zero rows with no padding to write, M == 0 or N == 0: OK without a launch
+    assert L.nvfp4_quantize(None, 0, 0, 64, 64, None, None, None, 0, 0, None) == 0
+    assert L.nvfp4_gemm(*([None] * 7), 0, 8, 0, 8, 64, None, 0, None) == 0
+    assert L.w4a4_gemm(None, 0, 64, None, None, None, None, None, 0, 8, 0, 8, 64, None, 0, None) == 0

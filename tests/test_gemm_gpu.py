@@ -1,0 +1,148 @@
+"""GPU parity of the block-scaled W4A4 GEMM (nvfp4_gemm) and of the whole
+linear layer (w4a4_gemm: on-the-fly activation quantize + GEMM) against the
+float64 CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_w4a4_quantized_06_b200 import native
+from nvfp4_w4a4_quantized_06_b200 import workloads as W
+from parity import assert_codes_equal, assert_gemm_close, f32, to_f32_numpy
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _quantized_weight(wl):
+    """Quantize (and for a fused group, harmonize) the workload's weight on the
+    GPU.  Returns (codes, sf, g*, per-module (cpu tensor, g))."""
+    K, N = wl.K, wl.N
+    offs = np.concatenate([[0], np.cumsum(wl.modules)]).astype(np.int64)
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=DEV)
+    sf = torch.empty(native.sf_bytes(N, K), dtype=torch.uint8, device=DEV)
+    mods = []
+    for m in range(len(wl.modules)):
+        w = W.make_w(wl, m)
+        wd = w.to(DEV)
+        g = native.amax_gscale(wd)
+        native.quantize(wd, g, codes=codes[offs[m]:offs[m + 1]], sf=sf, sf_row0=int(offs[m]), sf_rows_total=N)
+        mods.append((w, g))
+    if len(mods) > 1:
+        gw = native.harmonize(sf, N, K, offs, torch.cat([g for _, g in mods]))
+    else:
+        gw = mods[0][1]
+    return codes, sf, gw, mods, offs
+
+
+def _oracle_weight_rows(wl, mods, offs, cols):
+    """Oracle codes/scales of the fused weight's rows `cols` (sorted), with the
+    same per-module scales and the same harmonization."""
+    K = wl.K
+    per = [cols[(cols >= offs[m]) & (cols < offs[m + 1])] - offs[m] for m in range(len(mods))]
+    sub_offs = np.concatenate([[0], np.cumsum([len(p) for p in per])])
+    sf = np.zeros(oracle.sf_bytes(int(sub_offs[-1]), K), np.uint8)
+    codes = []
+    for m, p in enumerate(per):
+        if len(p):
+            c, _ = oracle.quantize(to_f32_numpy(mods[m][0][torch.from_numpy(p)]), f32(mods[m][1]),
+                                   sf=sf, sf_row0=int(sub_offs[m]))
+            codes.append(c)
+    gs = [f32(g) for _, g in mods]
+    if len(mods) > 1:
+        keep = [m for m, p in enumerate(per) if len(p)]
+        gstar = oracle.harmonize(sf, K, sub_offs, gs) if len(keep) == len(mods) else None
+        assert gstar is not None, "sample every module"
+    else:
+        gstar = gs[0]
+    return np.concatenate(codes), sf, gstar
+
+
+def _run_linear(wl, out_dtype, rows=None, cols=None):
+    x_cpu = W.make_x(wl)
+    x = x_cpu.to(DEV)
+    gx = native.amax_gscale(x)
+    codes, sf, gw, mods, offs = _quantized_weight(wl)
+    y = native.linear(x, gx, codes, sf, gw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+    rows = np.arange(wl.M) if rows is None else rows
+    cols = np.arange(wl.N) if cols is None else cols
+    wc, ws, gstar = _oracle_weight_rows(wl, mods, offs, cols)
+    assert f32(gw) == gstar
+    y_ref, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu[torch.from_numpy(rows)]),
+                                                f32(gx), wc, ws, gstar)
+    yg = y[torch.from_numpy(rows).to(DEV)][:, torch.from_numpy(cols).to(DEV)]
+    return assert_gemm_close(yg, y_ref, yabs)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_tiny_linear(out_dtype):
+    _run_linear(W.WORKLOADS["tiny"], out_dtype)
+
+
+def _random_case(M, N, K, seed, out_dtype, a_dtype=torch.bfloat16):
+    x_cpu = W.gaussian(M, K, seed=seed, outliers=W.Outliers("scale", 0.02, 30.0), dtype=a_dtype)
+    w_cpu = W.gaussian(N, K, seed=seed + 1, std=0.02, dtype=a_dtype)
+    x, w = x_cpu.to(DEV), w_cpu.to(DEV)
+    gx, gw = native.amax_gscale(x), native.amax_gscale(w)
+    ac, asf = native.quantize(x, gx)
+    bc, bsf = native.quantize(w, gw)
+    y = native.gemm(ac, asf, gx, bc, bsf, gw, out_dtype=out_dtype)
+    y2 = native.linear(x, gx, bc, bsf, gw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+    rc, rs = oracle.quantize(to_f32_numpy(x_cpu), f32(gx))
+    wc, ws = oracle.quantize(to_f32_numpy(w_cpu), f32(gw))
+    assert_codes_equal(ac, rc)
+    y_ref, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu), f32(gx), wc, ws, f32(gw))
+    e = assert_gemm_close(y, y_ref, yabs)
+    assert torch.equal(y, y2)          # linear == quantize + gemm, bit for bit
+    return e
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 256),      # one tile, one stage
+    (256, 512, 1024),     # several tiles and stages
+    (200, 300, 320),      # ragged M and N, K not a multiple of 256
+    (129, 96, 5120),      # small N (128-wide tile), split-K
+    (384, 1000, 1344),    # ragged everything, several waves of stages
+])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_shapes(M, N, K, out_dtype):
+    _random_case(M, N, K, seed=M + N + K, out_dtype=out_dtype)
+
+
+@pytest.mark.parametrize("M", [1, 7, 32, 33, 64])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_decode_shapes(M, out_dtype):
+    """M <= 64 runs the weight through the 128-row MMA side with split-K."""
+    _random_case(M, 640, 2048, seed=M, out_dtype=out_dtype)
+
+
+def test_gemm_fp32_activation():
+    _random_case(96, 128, 512, seed=5, out_dtype=torch.float32, a_dtype=torch.float32)
+
+
+def test_gdn_gates_fused_group():
+    _run_linear(W.WORKLOADS["gdn_gates_ab"], torch.float32, rows=W.sample_rows(4096, 512))
+
+
+@pytest.mark.parametrize("name", ["decode_out_proj", "decode_down_proj"])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_decode_workloads(name, out_dtype):
+    _run_linear(W.WORKLOADS[name], out_dtype, cols=W.sample_rows(5120, 640))
+
+
+def test_gdn_qkv_z_fused_group():
+    wl = W.WORKLOADS["gdn_qkv_z"]
+    cols = np.unique(np.concatenate([W.sample_rows(10240, 200, seed=3),
+                                     10240 + W.sample_rows(6144, 200, seed=4)]))
+    _run_linear(wl, torch.bfloat16, rows=W.sample_rows(wl.M, 96), cols=cols)
+
+
+def test_prefill_mlp_full_size():
+    """The full 32768 x 34816 x 5120 product in the launch configuration the
+    benchmark times, checked on a seeded sample of outputs."""
+    wl = W.WORKLOADS["prefill_mlp_gate_up"]
+    _run_linear(wl, torch.bfloat16, rows=W.sample_rows(wl.M, 64), cols=W.sample_rows(wl.N, 512, seed=9))
