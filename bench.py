@@ -207,7 +207,7 @@ def run_native(args, rank, world, dev):
     q_gbs = quant_bytes(M, K) / (tq_ms * 1e-3) / 1e9
 
     # ---- end to end through the public one-call API, host buffers
-    e2e = measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world)
+    e2e = None if args.no_e2e else measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world)
 
     also = {}
     if world == 1 and not args.headline_only:
@@ -426,6 +426,7 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--headline-only", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

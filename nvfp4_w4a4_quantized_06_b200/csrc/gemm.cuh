@@ -19,11 +19,10 @@
 //   warps 2..   epilogue: tcgen05.ld the FP32 accumulator (lane = row i), hand
 //               TMEM back as soon as it is in registers, then scale, convert
 //               and store while the next tile's MMAs run.
-// TMEM columns: [0, BN) accumulator, then 16 columns of A scales (4 MMAs x 4
-// columns) and 16*BN/128 columns of B scales.  The scale region is rewritten
-// every stage; tcgen05.cp and tcgen05.mma issued by one thread execute in
-// issue order, so the copy for stage k+1 lands after the MMAs of stage k have
-// read their scales.
+// TMEM columns: [0, BN) accumulator, then one scale region per pipeline stage
+// (16 columns of A scales, 4 MMAs x 4 columns, and 16*BN/128 of B scales).  A
+// region is rewritten only after the producer has refilled its stage, i.e.
+// after the MMAs that read it have completed.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -63,9 +62,12 @@ struct GemmCfg {
   static constexpr int EPI_WARPS = BN >= 64 ? 8 : 4;
   static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);   // columns per epilogue warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // per-stage scale-factor regions after the accumulator: A scales (4 MMAs x 4
+  // columns) then B scales (4 MMAs x 4 columns per 128 rows)
+  static constexpr int SF_COLS = 16 + 16 * SFB_ATOMS;
   static constexpr int SFA_COL = BN;
   static constexpr int SFB_COL = BN + 16;
-  static constexpr int TMEM_NEEDED = BN + 16 + 16 * SFB_ATOMS;
+  static constexpr int TMEM_NEEDED = BN + STAGES * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_NEEDED <= 32 ? 32 : TMEM_NEEDED <= 64 ? 64
                                   : TMEM_NEEDED <= 128 ? 128 : TMEM_NEEDED <= 256 ? 256 : 512;
   static constexpr int BAR_BYTES = 256;
@@ -233,36 +235,59 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------- MMA issue
+      // One thread feeds the tensor pipe, so this loop is kept lean: every
+      // descriptor is built once and advanced by immediate adds (the start
+      // address sits in the low 14 bits, addresses stay below 256 KB), and the
+      // four K-blocks of a stage are unrolled.  Per K-block the scale atoms are
+      // copied into this stage's TMEM region right before the MMA that reads
+      // them; stages rotate through their own regions.
+      const uint64_t a_desc0 = smem_desc(smem_u32(sA), 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(smem_u32(sB), 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(smem_u32(sSFA), 0, 128, 0);
+      const uint64_t sfb_desc0 = smem_desc(smem_u32(sSFB), 0, 128, 0);
       int st = 0;
       uint32_t ph = 0;
       int it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++it) {
+      for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++it) {
         int ta, tb, split, ks0, ks1;
         unit_coords(p, u, ta, tb, split);
         split_range(p, split, ks0, ks1);
-        if (!mbar_wait(tempty, (it & 1) ^ 1, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(tempty, (it & 1) ^ 1, p.err, ERR_MMA, abort_flag)) break;
         tc_fence_after();
+        bool ok = true;
         for (int ks = ks0; ks < ks1; ++ks) {
           if (!mbar_wait(&full[st], ph, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const int nkb = min(4, p.kblocks - ks * 4);
-          const uint32_t a_base = smem_u32(sA + st * C::A_BYTES);
-          const uint32_t b_base = smem_u32(sB + st * C::B_BYTES);
-          const uint32_t sfa_base = smem_u32(sSFA + st * C::SFA_BYTES);
-          const uint32_t sfb_base = smem_u32(sSFB + st * C::SFB_BYTES);
-          for (int kb = 0; kb < nkb; ++kb) {
-            tc_cp_32x128b_warpx4(tmem + C::SFA_COL + 4 * kb, smem_desc(sfa_base + kb * 512, 0, 128, 0));
+          const uint64_t ad = a_desc0 + (uint64_t)((st * C::A_BYTES) >> 4);
+          const uint64_t bd = b_desc0 + (uint64_t)((st * C::B_BYTES) >> 4);
+          const uint64_t sad = sfa_desc0 + (uint64_t)((st * C::SFA_BYTES) >> 4);
+          const uint64_t sbd = sfb_desc0 + (uint64_t)((st * C::SFB_BYTES) >> 4);
+          const uint32_t reg = tmem + (uint32_t)(st * C::SF_COLS);
+          const uint32_t acc0 = ks > ks0 ? 1u : 0u;
+          if (ks * 4 + 4 <= p.kblocks) {
 #pragma unroll
-            for (int j = 0; j < C::SFB_ATOMS; ++j)
-              tc_cp_32x128b_warpx4(tmem + C::SFB_COL + kb * 4 * C::SFB_ATOMS + 4 * j,
-                                   smem_desc(sfb_base + j * 2048 + kb * 512, 0, 128, 0));
-          }
-          for (int kb = 0; kb < nkb; ++kb) {
-            const uint64_t ad = smem_desc(a_base + kb * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_base + kb * 32, 16, 1024, 2);
-            tc_mma_nvfp4(tmem, ad, bd, C::IDESC, (ks > ks0 || kb > 0) ? 1u : 0u,
-                         tmem + C::SFA_COL + 4 * kb, tmem + C::SFB_COL + kb * 4 * C::SFB_ATOMS);
+            for (int kb = 0; kb < 4; ++kb) {
+              tc_cp_32x128b_warpx4(reg + C::SFA_COL + 4 * kb, sad + (uint64_t)(kb * 32));
+#pragma unroll
+              for (int j = 0; j < C::SFB_ATOMS; ++j)
+                tc_cp_32x128b_warpx4(reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS + 4 * j,
+                                     sbd + (uint64_t)(j * 128 + kb * 32));
+              tc_mma_nvfp4(tmem, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), C::IDESC,
+                           kb > 0 ? 1u : acc0, reg + C::SFA_COL + 4 * kb,
+                           reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS);
+            }
+          } else {
+            const int nkb = p.kblocks - ks * 4;      // K tail: 1 to 3 blocks
+            for (int kb = 0; kb < nkb; ++kb) {
+              tc_cp_32x128b_warpx4(reg + C::SFA_COL + 4 * kb, sad + (uint64_t)(kb * 32));
+#pragma unroll
+              for (int j = 0; j < C::SFB_ATOMS; ++j)
+                tc_cp_32x128b_warpx4(reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS + 4 * j,
+                                     sbd + (uint64_t)(j * 128 + kb * 32));
+              tc_mma_nvfp4(tmem, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), C::IDESC,
+                           kb > 0 ? 1u : acc0, reg + C::SFA_COL + 4 * kb,
+                           reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS);
+            }
           }
           tc_commit(&empty[st]);
           if (++st == C::STAGES) { st = 0; ph ^= 1; }

@@ -244,6 +244,14 @@ nvfp4_status check_gemm_args(const uint8_t *a_codes, const uint8_t *a_sf, const 
 
 template <typename T>
 void launch_quantize(const QuantizeParams &p, int sms, cudaStream_t s) {
+  const bool tile_ok = (p.sf_row0 % 128) == 0 && ((p.rows % 128) == 0 || p.pad_rows > 0 || p.rows == 0);
+  if (tile_ok && p.rows > 0) {
+    constexpr int U = sizeof(T) == 2 ? 8 : 4;
+    const int64_t units = ((p.rows + 127) / 128) * ((p.K + 255) / 256);
+    int64_t blocks = units < 4LL * sms ? units : 4LL * sms;
+    quantize_tile_kernel<T, U><<<(unsigned)blocks, 256, 0, s>>>(p);
+    return;
+  }
   constexpr int U = 4;
   const int64_t nseg = (p.K + 255) / 256;
   const int64_t units = p.rows * nseg;
@@ -300,7 +308,8 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int6
                             const float *gscale, uint8_t *codes, uint8_t *sf, int64_t sf_row0,
                             int64_t sf_rows_total, nvfp4_stream_t stream) {
   if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
-  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || sf_row0 < 0 || sf_rows_total < sf_row0 + rows)
+  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || sf_row0 < 0 || sf_rows_total < sf_row0 + rows ||
+      rows * ((K + 255) / 256) >= (int64_t)UINT32_MAX)
     return NVFP4_ERR_SHAPE;
   const bool owns_pad = sf_row0 + rows == sf_rows_total;
   const int64_t pad_rows = owns_pad ? pad128(sf_rows_total) - sf_rows_total : 0;

@@ -29,6 +29,7 @@ struct Vec8;  // eight consecutive input elements as fp32
 template <>
 struct Vec8<__nv_bfloat16> {
   uint4 raw;
+  __device__ __forceinline__ void zero() { raw = make_uint4(0u, 0u, 0u, 0u); }
   __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
     raw = __ldg(reinterpret_cast<const uint4 *>(p));
   }
@@ -45,6 +46,10 @@ struct Vec8<__nv_bfloat16> {
 template <>
 struct Vec8<float> {
   float4 a, b;
+  __device__ __forceinline__ void zero() {
+    a = make_float4(0.f, 0.f, 0.f, 0.f);
+    b = a;
+  }
   __device__ __forceinline__ void load(const float *p) {
     a = __ldg(reinterpret_cast<const float4 *>(p));
     b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
@@ -57,6 +62,15 @@ struct Vec8<float> {
 
 // Encode eight values of one half-block given the block's amax; returns the
 // packed code word and (through *s_out) the E4M3 scale byte.
+//
+// The codes must equal E2M1(fl32(x/d)) exactly.  Fast path: y = fl32(x * r)
+// with r = fl32(1/d) (correctly rounded reciprocal) differs from fl32(x/d) by
+// at most 3 ulps.  The E2M1 code can only differ between two values if one of
+// the decision thresholds 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 lies between
+// them; every threshold has 21 trailing zero bits in its fp32 encoding, so a
+// |y| whose bit pattern is within 8 of a multiple of 2^21 (and |y| >= 0.125)
+// is the only case that can be affected.  Those groups, and any block whose d
+// or 1/d is not a normal number, take the IEEE division.
 __device__ __forceinline__ uint32_t encode8(const float (&v)[8], float amax, float g, float g6,
                                             uint32_t *s_out) {
   const float t = __fdiv_rn(amax, g6);
@@ -65,9 +79,19 @@ __device__ __forceinline__ uint32_t encode8(const float (&v)[8], float amax, flo
   const float d = __fmul_rn(decs, g);
   *s_out = s;
   if (decs == 0.0f || d == 0.0f) return 0u;
+  const float r = __frcp_rn(d);
+  bool exact = d >= 1.17549435e-38f && r >= 1.17549435e-38f && r <= 3.40282347e38f;
   float y[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(v[i], d);
+  for (int i = 0; i < 8; ++i) {
+    y[i] = __fmul_rn(v[i], r);
+    const uint32_t b = __float_as_uint(y[i]) & 0x7FFFFFFFu;
+    exact = exact && (((b + 8u) & 0x1FFFF0u) != 0u || b < 0x3E000000u);
+  }
+  if (!exact) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(v[i], d);
+  }
   return f32x8_to_e2m1(y);
 }
 
@@ -81,48 +105,50 @@ struct QuantizeParams {
   int64_t pad_rows;  // padding rows (zeroed) after this call's rows, or 0
 };
 
-// One warp handles a 256-element segment of one row per unit: lane l owns
-// elements [8l, 8l+8), lanes 2i and 2i+1 form 16-element block i and exchange
-// their half-maxima with one shuffle.  Loads are 16-byte vectors (a warp reads
-// 512 contiguous bytes of bf16), code words are 4-byte stores (128 contiguous
-// bytes per warp).  UNROLL units are loaded before any is encoded.
+// Generic path (any row offset inside a fused buffer): one warp handles a
+// 256-element segment of one row per unit; lane l owns elements [8l, 8l+8),
+// lanes 2i and 2i+1 form 16-element block i and exchange their half-maxima
+// with one shuffle.  Loads are 16-byte vectors, code words 4-byte stores, and
+// every scale byte is stored on its own.  UNROLL units are loaded before any
+// is encoded.
 template <typename T, int UNROLL>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantizeParams p) {
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t nseg = (p.K + 255) >> 8;
-  const int64_t units = p.rows * nseg;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t nseg = (uint32_t)((p.K + 255) >> 8);
+  const uint32_t units = (uint32_t)p.rows * nseg;
   const int64_t ncols = p.K >> 4;
   const float g = __ldg(p.gscale);
   const float g6 = __fmul_rn(6.0f, g);
   const T *x = static_cast<const T *>(p.x);
 
-  for (int64_t u0 = warp * UNROLL; u0 < units; u0 += nwarps * UNROLL) {
+  for (uint32_t u0 = warp * UNROLL; u0 < units; u0 += nwarps * UNROLL) {
     Vec8<T> in[UNROLL];
+    int64_t row[UNROLL];
+    int col[UNROLL];
 #pragma unroll
     for (int j = 0; j < UNROLL; ++j) {
-      const int64_t u = u0 + j;
-      const int64_t row = u / nseg, col = (u - row * nseg) * 256 + lane * 8;
-      if (u < units && col < p.K) in[j].load(x + row * p.ld_x + col);
+      const uint32_t u = u0 + j;
+      row[j] = u / nseg;
+      col[j] = (int)(u - (uint32_t)row[j] * nseg) * 256 + lane * 8;
+      in[j].zero();
+      if (u < units && col[j] < p.K) in[j].load(x + row[j] * p.ld_x + col[j]);
     }
 #pragma unroll
     for (int j = 0; j < UNROLL; ++j) {
-      const int64_t u = u0 + j;
-      const int64_t row = u / nseg, col = (u - row * nseg) * 256 + lane * 8;
-      const bool active = u < units && col < p.K;
+      const bool active = u0 + j < units && col[j] < p.K;
       float v[8];
       in[j].to_f32(v);
       float amax = 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      if (!active) amax = 0.0f;
       amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
       if (active) {
         uint32_t s;
         const uint32_t word = encode8(v, amax, g, g6, &s);
-        *reinterpret_cast<uint32_t *>(p.codes + row * (p.K >> 1) + (col >> 1)) = word;
-        if ((lane & 1) == 0) p.sf[sf_index(p.sf_row0 + row, col >> 4, p.K)] = static_cast<uint8_t>(s);
+        *reinterpret_cast<uint32_t *>(p.codes + row[j] * (p.K >> 1) + (col[j] >> 1)) = word;
+        if ((lane & 1) == 0) p.sf[sf_index(p.sf_row0 + row[j], col[j] >> 4, p.K)] = static_cast<uint8_t>(s);
       }
     }
   }
@@ -133,6 +159,69 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantizeParams p) {
   for (int64_t i = tid; i < pad_bytes; i += nthreads) {
     const int64_t r = p.sf_row0 + p.rows + i / ncols, c = i % ncols;
     p.sf[sf_index(r, c, p.K)] = 0;
+  }
+}
+
+// Tile path, used when this call's scale rows start on a 128-row boundary and
+// it owns every row of its last 128-row block (the activation quantize always
+// does).  A CTA of 8 warps handles a 128-row x 256-column tile: warp w encodes
+// rows w, w+8, ..., w+120 of the tile (each lane 8 elements per row, 512
+// contiguous input bytes per warp-row), collects the tile's 16 scale columns
+// in shared memory -- exactly four 512-byte atoms, contiguous in the swizzled
+// buffer -- and the CTA writes them with 16-byte stores.  Rows past `rows`
+// (padding) get zero scales.
+template <typename T, int UNROLL>
+__global__ void __launch_bounds__(256) quantize_tile_kernel(QuantizeParams p) {
+  __shared__ __align__(16) uint8_t sf_tile[2048];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t nseg = (uint32_t)((p.K + 255) >> 8);
+  const uint32_t nrb = (uint32_t)((p.rows + 127) >> 7);
+  const uint32_t units = nrb * nseg;
+  const uint32_t atoms_per_rb = (uint32_t)(p.K >> 6);
+  const float g = __ldg(p.gscale);
+  const float g6 = __fmul_rn(6.0f, g);
+  const T *x = static_cast<const T *>(p.x);
+  const int c_in_seg = lane >> 1;                 // 16-element block inside the segment
+
+  for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const uint32_t rb = u / nseg, seg = u - rb * nseg;
+    const int col = (int)seg * 256 + lane * 8;
+    const bool col_ok = col < p.K;
+#pragma unroll 1
+    for (int i0 = 0; i0 < 16; i0 += UNROLL) {
+      Vec8<T> in[UNROLL];
+#pragma unroll
+      for (int j = 0; j < UNROLL; ++j) {
+        const int64_t row = (int64_t)rb * 128 + warp + 8 * (i0 + j);
+        in[j].zero();
+        if (col_ok && row < p.rows) in[j].load(x + row * p.ld_x + col);
+      }
+#pragma unroll
+      for (int j = 0; j < UNROLL; ++j) {
+        const int rl = warp + 8 * (i0 + j);
+        const int64_t row = (int64_t)rb * 128 + rl;
+        float v[8];
+        in[j].to_f32(v);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        uint32_t s = 0;
+        if (col_ok && row < p.rows) {
+          const uint32_t word = encode8(v, amax, g, g6, &s);
+          *reinterpret_cast<uint32_t *>(p.codes + row * (p.K >> 1) + (col >> 1)) = word;
+        }
+        if ((lane & 1) == 0)
+          sf_tile[(c_in_seg >> 2) * 512 + (rl & 31) * 16 + (rl >> 5) * 4 + (c_in_seg & 3)] = (uint8_t)s;
+      }
+    }
+    __syncthreads();
+    const uint32_t natoms = min(4u, atoms_per_rb - seg * 4);
+    if (threadIdx.x < natoms * 32) {
+      uint8_t *dst = p.sf + ((int64_t)((p.sf_row0 >> 7) + rb) * atoms_per_rb + seg * 4) * 512;
+      reinterpret_cast<uint4 *>(dst)[threadIdx.x] = reinterpret_cast<const uint4 *>(sf_tile)[threadIdx.x];
+    }
+    __syncthreads();
   }
 }
 
