@@ -31,6 +31,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 0;
   unsigned *err = nullptr;
+  int qtile_bf16 = 1, qtile_f32 = 1;   // resident quantize-tile CTAs per SM
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -77,6 +78,13 @@ nvfp4_status device_state(DeviceState **out) {
     if (set_gemm_attrs<256>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
         set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<32>() != cudaSuccess)
       return NVFP4_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qtile_bf16, quantize_tile_kernel<__nv_bfloat16, 4>, 256, 0) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qtile_f32, quantize_tile_kernel<float, 4>, 256, 0) !=
+            cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    if (d.qtile_bf16 < 1) d.qtile_bf16 = 1;
+    if (d.qtile_f32 < 1) d.qtile_f32 = 1;
     d.sms = sms;
     d.err = static_cast<unsigned *>(errp);
     d.ready = true;
@@ -243,20 +251,22 @@ nvfp4_status check_gemm_args(const uint8_t *a_codes, const uint8_t *a_sf, const 
 }
 
 template <typename T>
-void launch_quantize(const QuantizeParams &p, int sms, cudaStream_t s) {
+void launch_quantize(const QuantizeParams &p, const DeviceState &dev, cudaStream_t s) {
   const bool tile_ok = (p.sf_row0 % 128) == 0 && ((p.rows % 128) == 0 || p.pad_rows > 0 || p.rows == 0);
   if (tile_ok && p.rows > 0) {
-    constexpr int U = sizeof(T) == 2 ? 8 : 4;
-    const int64_t units = ((p.rows + 127) / 128) * ((p.K + 255) / 256);
-    int64_t blocks = units < 4LL * sms ? units : 4LL * sms;
-    quantize_tile_kernel<T, U><<<(unsigned)blocks, 256, 0, s>>>(p);
+    // one wave of resident CTAs, each looping over 128-row x 512-column tiles
+    const int per_sm = sizeof(T) == 2 ? dev.qtile_bf16 : dev.qtile_f32;
+    const int64_t units = ((p.rows + 127) / 128) * ((p.K + 511) / 512);
+    const int64_t wave = (int64_t)per_sm * dev.sms;
+    const int64_t blocks = units < wave ? units : wave;
+    quantize_tile_kernel<T, 4><<<(unsigned)blocks, 256, 0, s>>>(p);
     return;
   }
   constexpr int U = 4;
   const int64_t nseg = (p.K + 255) / 256;
   const int64_t units = p.rows * nseg;
   int64_t blocks = ((units + U - 1) / U + 7) / 8;
-  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  if (blocks > 8LL * dev.sms) blocks = 8LL * dev.sms;
   if (blocks < 1) blocks = 1;
   quantize_kernel<T, U><<<(unsigned)blocks, 256, 0, s>>>(p);
 }
@@ -322,8 +332,8 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int6
   if (st != NVFP4_OK) return st;
   QuantizeParams p{x, rows, K, ld_x, gscale, codes, sf, sf_row0, pad_rows};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dt == NVFP4_IN_BF16) launch_quantize<__nv_bfloat16>(p, dev->sms, s);
-  else launch_quantize<float>(p, dev->sms, s);
+  if (dt == NVFP4_IN_BF16) launch_quantize<__nv_bfloat16>(p, *dev, s);
+  else launch_quantize<float>(p, *dev, s);
   return launched();
 }
 
