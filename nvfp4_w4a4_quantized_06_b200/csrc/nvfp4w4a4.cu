@@ -14,6 +14,7 @@
 #include "ptx.cuh"
 #include "quantize.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 
 using namespace nvfp4;
 
@@ -32,6 +33,7 @@ struct DeviceState {
   int sms = 0;
   unsigned *err = nullptr;
   int qtile_bf16 = 1, qtile_f32 = 1;   // resident quantize-tile CTAs per SM
+  int pair_clusters = 0;                // co-resident CTA pairs of the pair GEMM
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -42,6 +44,13 @@ inline size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+cudaError_t set_pair_attrs() {
+  const int b = PairCfg::SMEM_BYTES;
+  cudaError_t e = set_smem(nvfp4_gemm_pair_kernel<OUT_BF16>, b);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_pair_kernel<OUT_F32>, b);
+  return e;
 }
 
 template <int BN>
@@ -76,8 +85,25 @@ nvfp4_status device_state(DeviceState **out) {
     void *errp = nullptr;
     if (cudaGetSymbolAddress(&errp, g_nvfp4_device_error) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (set_gemm_attrs<256>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
-        set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<32>() != cudaSuccess)
+        set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<32>() != cudaSuccess ||
+        set_pair_attrs() != cudaSuccess)
       return NVFP4_ERR_CUDA;
+    {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * sms);
+      cfg.blockDim = dim3(PairCfg::THREADS);
+      cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&d.pair_clusters, nvfp4_gemm_pair_kernel<OUT_BF16>, &cfg) != cudaSuccess)
+        d.pair_clusters = 0;
+      cudaGetLastError();
+    }
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qtile_bf16, quantize_tile_kernel<__nv_bfloat16, 4>, 256, 0) !=
             cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qtile_f32, quantize_tile_kernel<float, 4>, 256, 0) !=
@@ -109,18 +135,46 @@ bool make_codes_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K,
   return r == CUDA_SUCCESS;
 }
 
+// The swizzled scale buffer viewed as uint64 [pad128(rows)/128][K]: one
+// "row" per 128-row block holds its K/64 atoms of 512 bytes; a box of 256
+// elements is the 2 KB (four atoms) of one 256-deep K stage.  Boxes past the
+// last row block or past K read zeros.
+bool make_sf_map(CUtensorMap *map, const void *sf, int64_t rows, int64_t K, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)(pad128(rows) / 128)};
+  cuuint64_t strides[1] = {(cuuint64_t)(K * 8)};
+  cuuint32_t box[2] = {256u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(sf), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // GEMM plan: which operand drives the 128-row MMA dimension, the tile width,
 // split-K and the grid.
 struct Plan {
+  bool pair;       // CTA-pair kernel, 256 x 256 tiles
   bool swap;       // A operand = weight (rows N), B operand = activation (rows M)
   int bn;
   int tiles_a, tiles_b, splits, kstages;
   int grid;
 };
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int sms) {
+Plan make_plan(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters) {
   Plan pl{};
   pl.kstages = (int)((K / 64 + 3) / 4);
+  if (M > 128 && N > 128 && pair_clusters > 0 &&
+      ((M + 255) / 256) * ((N + 255) / 256) >= pair_clusters) {
+    // large products: CTA pairs on 256 x 256 tiles, one wave of resident pairs
+    pl.pair = true;
+    pl.bn = 256;
+    pl.tiles_a = (int)((M + 255) / 256);
+    pl.tiles_b = (int)((N + 255) / 256);
+    pl.splits = 1;
+    const int units = pl.tiles_a * pl.tiles_b;
+    pl.grid = 2 * (units < pair_clusters ? units : pair_clusters);
+    return pl;
+  }
   if (M <= 64) {
     // decode-shaped: the weight streams through the 128-row MMA dimension and
     // the few activation rows are the MMA's N; split K so that every SM
@@ -147,15 +201,15 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sms) {
   return pl;
 }
 
-size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, int sms) {
-  const Plan pl = make_plan(M, N, K, sms);
+size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters) {
+  const Plan pl = make_plan(M, N, K, sms, pair_clusters);
   return pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
 }
 
-int current_sms() {
+size_t current_partial_bytes(int64_t M, int64_t N, int64_t K) {
   DeviceState *d = nullptr;
-  if (device_state(&d) != NVFP4_OK) return 148;
-  return d->sms;
+  if (device_state(&d) != NVFP4_OK) return gemm_partial_bytes(M, N, K, 148, 0);
+  return gemm_partial_bytes(M, N, K, d->sms, d->pair_clusters);
 }
 
 template <int BN>
@@ -179,10 +233,50 @@ nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   nvfp4_status st = device_state(&dev);
   if (st != NVFP4_OK) return st;
   if (M == 0 || N == 0) return NVFP4_OK;
-  const Plan pl = make_plan(M, N, K, dev->sms);
+  const Plan pl = make_plan(M, N, K, dev->sms, dev->pair_clusters);
   const size_t need = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
   if (need > 0 && (ws == nullptr || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
   if (need > 0 && !aligned16(ws)) return NVFP4_ERR_ALIGN;
+
+  if (pl.pair) {
+    GemmParams p{};
+    p.ga = a_gscale;
+    p.gb = b_gscale;
+    p.rows_a = (int)M;
+    p.rows_b = (int)N;
+    p.K = (int)K;
+    p.kblocks = (int)(K / 64);
+    p.kstages = pl.kstages;
+    p.tiles_a = pl.tiles_a;
+    p.tiles_b = pl.tiles_b;
+    p.splits = 1;
+    p.group = 8;
+    p.err = dev->err;
+    p.out = y;
+    p.out_si = ld_y;
+    p.out_sj = 1;
+    CUtensorMap ma, mb, msa, msb;
+    if (!make_codes_map(&ma, a_codes, M, K, 128) || !make_codes_map(&mb, b_codes, N, K, 128) ||
+        !make_sf_map(&msa, a_sf, M, K, 1) || !make_sf_map(&msb, b_sf, N, K, 2))
+      return NVFP4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(PairCfg::THREADS);
+    cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = y_dt == NVFP4_OUT_BF16
+                        ? cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_BF16>, ma, mb, msa, msb, p)
+                        : cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_F32>, ma, mb, msa, msb, p);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    return launched();
+  }
 
   GemmParams p{};
   const uint8_t *op_a = pl.swap ? b_codes : a_codes;   // A = 128-row MMA operand
@@ -368,7 +462,7 @@ nvfp4_status nvfp4_harmonize_group(uint8_t *sf, int64_t rows_total, int64_t K, i
 
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
-  return gemm_partial_bytes(M, N, K, current_sms());
+  return current_partial_bytes(M, N, K);
 }
 
 nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
@@ -384,7 +478,7 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float
 size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
   return align256(nvfp4_codes_bytes(M, K)) + align256(nvfp4_sf_bytes(M, K)) +
-         gemm_partial_bytes(M, N, K, current_sms());
+         current_partial_bytes(M, N, K);
 }
 
 nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
@@ -408,7 +502,8 @@ nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const f
   if (st != NVFP4_OK) return st;
   DeviceState *dev = nullptr;
   if ((st = device_state(&dev)) != NVFP4_OK) return st;
-  if (workspace_bytes < codes_b + sf_b + gemm_partial_bytes(M, N, K, dev->sms)) return NVFP4_ERR_WORKSPACE;
+  if (workspace_bytes < codes_b + sf_b + gemm_partial_bytes(M, N, K, dev->sms, dev->pair_clusters))
+    return NVFP4_ERR_WORKSPACE;
   st = nvfp4_quantize(x, x_dt, M, K, ld_x, x_gscale, a_codes, a_sf, 0, M, stream);
   if (st != NVFP4_OK) return st;
   return gemm_impl(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K,

@@ -113,6 +113,30 @@ def test_gemm_shapes(M, N, K, out_dtype):
     _random_case(M, N, K, seed=M + N + K, out_dtype=out_dtype)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (4200, 4396, 1344),   # CTA-pair path: last row tile's second CTA past M, N and K tails
+    (2304, 2560, 5120),   # CTA-pair path, exact tiles
+])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_pair_shapes(M, N, K, out_dtype):
+    """Shapes with at least a full wave of 256 x 256 tiles run on CTA pairs."""
+    x_cpu = W.gaussian(M, K, seed=M, outliers=W.Outliers("scale", 0.02, 30.0))
+    w_cpu = W.gaussian(N, K, seed=N, std=0.02)
+    x, w = x_cpu.to(DEV), w_cpu.to(DEV)
+    gx, gw = native.amax_gscale(x), native.amax_gscale(w)
+    ac, asf = native.quantize(x, gx)
+    bc, bsf = native.quantize(w, gw)
+    y = native.gemm(ac, asf, gx, bc, bsf, gw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+    rows = W.sample_rows(M, 160, seed=3)
+    rows = np.unique(np.concatenate([rows, np.arange(M - 130, M)]))      # the ragged last tile
+    cols = np.unique(np.concatenate([W.sample_rows(N, 300, seed=4), np.arange(N - 60, N)]))
+    wc, ws = oracle.quantize(to_f32_numpy(w_cpu[torch.from_numpy(cols)]), f32(gw))
+    y_ref, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu[torch.from_numpy(rows)]), f32(gx), wc, ws, f32(gw))
+    assert_gemm_close(y[torch.from_numpy(rows).to(DEV)][:, torch.from_numpy(cols).to(DEV)], y_ref, yabs)
+
+
 @pytest.mark.parametrize("M", [1, 7, 32, 33, 64])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_gemm_decode_shapes(M, out_dtype):
