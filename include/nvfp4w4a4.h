@@ -72,7 +72,8 @@ typedef enum {
     NVFP4_ERR_UNSUPPORTED = 5, /* valid request this build does not serve */
     NVFP4_ERR_TIMEOUT = 6,     /* a kernel wait ran out (see nvfp4_last_device_status) */
     NVFP4_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
-    NVFP4_ERR_WORKSPACE = 8    /* workspace NULL or smaller than the size helper says */
+    NVFP4_ERR_WORKSPACE = 8,   /* workspace NULL or smaller than the size helper says */
+    NVFP4_ERR_SCRATCH_LIMIT = 9 /* w4a4_gemm_noalloc: the problem needs more scratch than its built-in buffer */
 } nvfp4_status;
 
 typedef enum { NVFP4_IN_BF16 = 0, NVFP4_IN_F32 = 1 } nvfp4_in_dtype;
@@ -171,6 +172,40 @@ nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const f
                        void *y, nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N,
                        int64_t K, void *workspace, size_t workspace_bytes,
                        nvfp4_stream_t stream);
+
+/*
+ * The W4A4 linear layer for callers that cannot allocate device memory: the
+ * same computation and kernels as w4a4_gemm, but the scratch it needs (the
+ * quantized activation and any split-K partial sums) lives in a fixed buffer
+ * inside the library instead of a caller-provided workspace.  No counterpart
+ * exists on the pages; this is a deployment convenience.
+ *
+ * Who needs it: host code that must not call cudaMalloc at the point of use,
+ * for example an inference runtime whose memory plan is fixed before serving
+ * starts (every device byte is owned by the framework's arena), a plugin that
+ * the host framework gives only input and output pointers, or code that has
+ * to stay free of allocation calls because an allocation can synchronize the
+ * device or fail under memory pressure in the middle of a step.
+ *
+ * The buffer is a file-scope 8 MiB (8,388,608-byte) __device__ array; every
+ * GPU that loads the library holds it until the process exits.  The arguments
+ * mean what they mean for w4a4_gemm; the caller still provides x, the
+ * weights, the scales and y.
+ *   - Problems whose w4a4_gemm_workspace_bytes(M, N, K) exceeds 8 MiB return
+ *     NVFP4_ERR_SCRATCH_LIMIT before anything is enqueued (decode-shaped
+ *     products, e.g. M <= 64 with N*K up to about 5120 x 17408, fit).
+ *   - The first call on a device looks the buffer's device address up
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one buffer, which keeps the last call's contents;
+ *     nothing in it has to start at zero.  Calls that can overlap on the GPU
+ *     (different streams, or different host threads) race on it: order them.
+ *   - Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                               const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale,
+                               void *y, nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N,
+                               int64_t K, nvfp4_stream_t stream);
 
 /*
  * Synchronizes the device, then reports and clears the library's device error

@@ -20,6 +20,11 @@ using namespace nvfp4;
 
 __device__ unsigned g_nvfp4_device_error;
 
+// Fixed scratch of w4a4_gemm_noalloc (see the header): quantized activation
+// and split-K partial sums for callers that cannot allocate.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -510,6 +515,33 @@ nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const f
                    a_sf + sf_b, workspace_bytes - codes_b - sf_b, reinterpret_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                               const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
+                               nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K,
+                               nvfp4_stream_t stream) {
+  // per-device address of the fixed scratch, looked up once with the device current
+  static std::mutex mu;
+  static void *scratch[kMaxDevices] = {};
+  if (x_dt != NVFP4_IN_BF16 && x_dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ld_x < K) return NVFP4_ERR_SHAPE;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  void *buf = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!scratch[dev]) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NVFP4_ERR_CUDA;
+      scratch[dev] = p;
+    }
+    buf = scratch[dev];
+  }
+  if (w4a4_gemm_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return NVFP4_ERR_SCRATCH_LIMIT;
+  return w4a4_gemm(x, x_dt, ld_x, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K, buf,
+                   kNoAllocScratchBytes, stream);
+}
+
 nvfp4_status nvfp4_last_device_status(int *flags) {
   if (!flags) return NVFP4_ERR_NULL;
   *flags = 0;
@@ -532,6 +564,7 @@ const char *nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_TIMEOUT: return "a kernel wait ran out";
     case NVFP4_ERR_CUDA: return "CUDA error";
     case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the 8 MiB built-in buffer of w4a4_gemm_noalloc";
   }
   return "unknown status";
 }

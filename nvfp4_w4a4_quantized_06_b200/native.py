@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(HERE, "libnvfp4w4a4.so")
 IN_BF16, IN_F32 = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 STATUS = {0: "ok", 1: "null pointer", 2: "bad shape", 3: "misaligned", 4: "bad dtype",
-          5: "unsupported", 6: "timeout", 7: "CUDA error", 8: "workspace"}
+          5: "unsupported", 6: "timeout", 7: "CUDA error", 8: "workspace", 9: "scratch limit"}
 
 _lib = None
 
@@ -46,11 +46,12 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, sz, vp]
         L.w4a4_gemm_workspace_bytes.argtypes, L.w4a4_gemm_workspace_bytes.restype = [i64, i64, i64], sz
         L.w4a4_gemm.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, sz, vp]
+        L.w4a4_gemm_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp]
         L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
-                  "w4a4_gemm", "nvfp4_last_device_status"):
+                  "w4a4_gemm", "w4a4_gemm_noalloc", "nvfp4_last_device_status"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -173,6 +174,23 @@ def linear(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf:
         _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
         _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _ptr(workspace), workspace.numel(),
         _stream()))
+    return out
+
+
+def linear_noalloc(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
+                   w_gscale: torch.Tensor, out_dtype=torch.bfloat16,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """The W4A4 linear without a caller workspace: the library's fixed 8 MiB
+    scratch buffer holds the quantized activation and split-K partials (for
+    callers that cannot allocate device memory at the point of use)."""
+    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check("w4a4_gemm_noalloc", lib().w4a4_gemm_noalloc(
+        _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
+        _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _stream()))
     return out
 
 

@@ -39,7 +39,7 @@ def test_size_helpers(L):
 
 
 def test_status_strings(L):
-    for s in range(9):
+    for s in range(10):
         assert L.nvfp4_status_string(s)
 
 
