@@ -116,7 +116,7 @@ def quantized_weight(wl, dev):
 
 def kernel_src_hash():
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "ptx.cuh", "nvfp4w4a4.cu"):
+    for f in ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh", "nvfp4w4a4.cu"):
         h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_06_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -235,7 +235,7 @@ def run_native(args, rank, world, dev):
         "quantize_frac_hbm": round(q_gbs / pk["hbm_gbs"], 3),
         "gemm_tflops": round(gemm_tflops, 1),
         "frac_fp4_spec": round(value / world / FP4_SPEC_TFLOPS, 3),
-        "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256,bf16>",
+        "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_pair_kernel<bf16>",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / fp4_peak, 3),
                      "peak_src": f"{pk['src']} bf16 burst x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
@@ -420,7 +420,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS))
