@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4w4a4.so")
 SOURCES = [os.path.join(CSRC, "nvfp4w4a4.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quantize.cuh", "gemm.cuh", "gemm_pair.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quantize.cuh", "gemm.cuh", "gemm_pair.cuh", "gemm_cluster.cuh")] + [
     os.path.join(ROOT, "include", "nvfp4w4a4.h")]
 
 

@@ -1,0 +1,307 @@
+// gemm_cluster.cuh -- block-scaled NVFP4 GEMM with split-K across the CTAs of
+// a thread-block cluster, reduced through distributed shared memory.
+//
+// Same product as gemm.cuh (D[i, j] = sum_k dec(A)[i, k] * dec(B)[j, k], FP32
+// accumulation; web pages on arXiv 2609.04098, ta-paperlens page, "前提1"),
+// for the shapes where one operand is narrow: decode (a few activation rows,
+// the weight on the 128-row MMA side) and small-N projections such as the
+// GDN a/b gates (N = 96).  Such products have too few 128-row tiles to fill
+// the GPU, so each tile is computed by a cluster of S CTAs, rank r taking
+// K stages [r*KS/S, (r+1)*KS/S):
+//   warp 0     TMA producer.  The loads of the operand that does not depend
+//              on the preceding kernel (the weight) are issued first, then
+//              the thread waits for that kernel (programmatic dependent
+//              launch) before loading the activation side.
+//   warp 1     TMEM allocation and MMA issue: tcgen05.cp of the scale atoms,
+//              four tcgen05.mma kind::mxf4nvf4 (K = 64) per stage.
+//   warps 2-5  epilogue: each CTA owns a share of the output tile (whole
+//              output columns for decode, whole rows otherwise); the FP32
+//              partial tile leaves TMEM and every element is stored straight
+//              into the owner CTA's shared memory, in the slot of the
+//              sending rank (fire-and-forget distributed-shared-memory
+//              stores).  After one cluster barrier each CTA sums its share
+//              over the S slots in rank order (so the result does not depend
+//              on timing), scales by fl32(g_a*g_b) and writes BF16 or FP32.
+// No partial sums touch global memory and no second kernel is launched.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+template <int BN>
+struct ClusterCfg {
+  static constexpr int BM = 128;
+  static constexpr int A_BYTES = BM * 128;                 // 256 FP4 per row per stage
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SFB_ATOMS = BN >= 128 ? BN / 128 : 1;
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_BYTES = SFB_ATOMS * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = BN <= 32 ? 8 : (BN <= 64 ? 6 : 4);
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int SF_COLS = 16 + 16 * SFB_ATOMS;
+  static constexpr int SFA_COL = BN;
+  static constexpr int SFB_COL = BN + 16;
+  static constexpr int TMEM_NEEDED = BN + STAGES * SF_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEEDED <= 64 ? 64 : TMEM_NEEDED <= 128 ? 128
+                                  : TMEM_NEEDED <= 256 ? 256 : 512;
+  static constexpr int MAX_SPLITS = 8;
+  // reduction slots: S slots, each one owner share: ceil(BN/S) columns of
+  // 128 floats, or ceil(128/S) rows of BN+1 floats (S * ceil(D/S) <= D+S-1)
+  static constexpr int RED_PITCH = BN + 1;                  // odd: conflict-free rows and columns
+  static constexpr int RED_NEED = (BN + MAX_SPLITS - 1) * BM > (BM + MAX_SPLITS - 1) * RED_PITCH
+                                      ? (BN + MAX_SPLITS - 1) * BM
+                                      : (BM + MAX_SPLITS - 1) * RED_PITCH;
+  static constexpr int RED_FLOATS = (RED_NEED + 31) / 32 * 32;   // keeps the barriers after it 128-byte aligned
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RED_FLOATS * 4 + 256;
+  static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                    ((uint32_t)(BM >> 4) << 24);
+  static_assert(BN % 16 == 0 && BN >= 32 && BN <= 128, "MMA N");
+  static_assert((STAGES * STAGE_BYTES + RED_FLOATS * 4) % 128 == 0, "mbarrier alignment");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(TMEM_NEEDED <= 512, "TMEM budget");
+};
+
+// p.splits = S (the cluster size), p.tiles_a x p.tiles_b tiles (one per
+// cluster), p.group != 0 when A is the operand independent of the preceding
+// kernel (the weight), 0 when B is.
+template <int BN, int MODE>
+__global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
+    nvfp4_gemm_cluster_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                              const GemmParams p) {
+  using C = ClusterCfg<BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + C::STAGES * C::A_BYTES;
+  uint8_t *sSFA = sB + C::STAGES * C::B_BYTES;
+  uint8_t *sSFB = sSFA + C::STAGES * C::SFA_BYTES;
+  float *red = reinterpret_cast<float *>(sSFB + C::STAGES * C::SFB_BYTES);   // reduction slots
+  uint64_t *bars = reinterpret_cast<uint64_t *>(red + C::RED_FLOATS);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + C::STAGES;
+  uint64_t *tfull = bars + 2 * C::STAGES;
+  uint64_t *tdone = tfull + 1;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tfull + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.splits;
+  const int rank = (int)cluster_ctarank();
+  const int tile = blockIdx.x / S;
+  const int ta = tile % p.tiles_a, tb = tile / p.tiles_a;
+  int ks0, ks1;
+  split_range(p, rank, ks0, ks1);
+  // output ownership: decode writes Y[m, n] with n = tile row i contiguous,
+  // so a CTA owns whole columns j; otherwise whole rows i
+  const bool i_fast = p.out_si == 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tdone, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tma);
+    prefetch_tmap(&tmb);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // the next kernel in the stream may be scheduled now; it waits for this
+  // grid's completion before it touches anything this grid reads or writes
+  if (threadIdx.x == 0) griddep_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      const int row_a = ta * C::BM, row_b = tb * BN;
+      const int pad_b = (p.rows_b + 127) & ~127;
+      const bool a_first = p.group != 0;
+      auto stage_bytes = [&](int ks) {
+        const int nkb = min(4, p.kblocks - ks * 4);
+        int nsfb = 0;
+#pragma unroll
+        for (int j = 0; j < C::SFB_ATOMS; ++j)
+          if (row_b + 128 * j < pad_b) ++nsfb;
+        return (uint32_t)(C::A_BYTES + C::B_BYTES) + (uint32_t)nkb * 512u * (1u + nsfb);
+      };
+      auto load_a = [&](int st, int ks) {
+        const int nkb = min(4, p.kblocks - ks * 4);
+        tma_load_2d(sA + st * C::A_BYTES, &tma, &full[st], ks * 128, row_a);
+        bulk_load(sSFA + st * C::SFA_BYTES, p.sfa + ((int64_t)(row_a >> 7) * p.kblocks + ks * 4) * 512,
+                  nkb * 512u, &full[st]);
+      };
+      auto load_b = [&](int st, int ks) {
+        const int nkb = min(4, p.kblocks - ks * 4);
+        tma_load_2d(sB + st * C::B_BYTES, &tmb, &full[st], ks * 128, row_b);
+#pragma unroll
+        for (int j = 0; j < C::SFB_ATOMS; ++j)
+          if (row_b + 128 * j < pad_b)
+            bulk_load(sSFB + st * C::SFB_BYTES + j * 2048,
+                      p.sfb + ((int64_t)((row_b >> 7) + j) * p.kblocks + ks * 4) * 512, nkb * 512u, &full[st]);
+      };
+      // the first ring's worth of stages: independent operand first, then
+      // wait for the preceding kernel, then the dependent operand
+      const int pre = min(ks1 - ks0, C::STAGES);
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], stage_bytes(ks0 + i));
+        if (a_first) load_a(i, ks0 + i); else load_b(i, ks0 + i);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) {
+        if (a_first) load_b(i, ks0 + i); else load_a(i, ks0 + i);
+      }
+      int st = pre == C::STAGES ? 0 : pre;
+      uint32_t ph = pre == C::STAGES ? 1u : 0u;
+      uint32_t issued = (uint32_t)pre;
+      for (int ks = ks0 + pre; ks < ks1; ++ks) {
+        if (!mbar_wait(&empty[st], ph ^ 1, p.err, ERR_PRODUCER, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[st], stage_bytes(ks));
+        load_a(st, ks);
+        load_b(st, ks);
+        ++issued;
+        if (++st == C::STAGES) { st = 0; ph ^= 1; }
+      }
+      // every armed stage's loads must have landed before the CTA exits
+      for (int s = 0; s < C::STAGES; ++s) {
+        const uint32_t armed = issued / C::STAGES + ((uint32_t)s < issued % C::STAGES ? 1u : 0u);
+        if (armed) {
+          volatile int never = 0;
+          mbar_wait(&full[s], (armed - 1) & 1, p.err, ERR_PRODUCER, &never);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------- MMA issue
+      const uint64_t a_desc0 = smem_desc(smem_u32(sA), 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(smem_u32(sB), 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(smem_u32(sSFA), 0, 128, 0);
+      const uint64_t sfb_desc0 = smem_desc(smem_u32(sSFB), 0, 128, 0);
+      int st = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        if (!mbar_wait(&full[st], ph, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t ad = a_desc0 + (uint64_t)((st * C::A_BYTES) >> 4);
+        const uint64_t bd = b_desc0 + (uint64_t)((st * C::B_BYTES) >> 4);
+        const uint64_t sad = sfa_desc0 + (uint64_t)((st * C::SFA_BYTES) >> 4);
+        const uint64_t sbd = sfb_desc0 + (uint64_t)((st * C::SFB_BYTES) >> 4);
+        const uint32_t reg = tmem + (uint32_t)(st * C::SF_COLS);
+        const int nkb = min(4, p.kblocks - ks * 4);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          if (kb < nkb) {
+            tc_cp_32x128b_warpx4(reg + C::SFA_COL + 4 * kb, sad + (uint64_t)(kb * 32));
+#pragma unroll
+            for (int j = 0; j < C::SFB_ATOMS; ++j)
+              tc_cp_32x128b_warpx4(reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS + 4 * j,
+                                   sbd + (uint64_t)(j * 128 + kb * 32));
+            tc_mma_nvfp4(tmem, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), C::IDESC,
+                         (ks > ks0 || kb > 0) ? 1u : 0u, reg + C::SFA_COL + 4 * kb,
+                         reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS);
+          }
+        }
+        tc_commit(&empty[st]);
+        if (++st == C::STAGES) { st = 0; ph ^= 1; }
+      }
+      if (ok) tc_commit(tfull);
+      // all issued tensor-core work must finish before TMEM is freed
+      tc_commit(tdone);
+      volatile int never = 0;
+      mbar_wait(tdone, 0, p.err, ERR_MMA, &never);
+    }
+  } else {
+    // ------------------------------- epilogue: partial tile -> owners' slots
+    const int q = warp & 3;                       // TMEM lane quarter of this warp
+    const int i = q * 32 + lane;                  // tile row (A row)
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const bool ok = mbar_wait(tfull, 0, p.err, ERR_EPILOGUE, abort_flag);
+    if (ok) tc_fence_after();
+    const uint32_t red_base = smem_u32(red);
+    // shares: index x of a dimension of size D belongs to rank x*S/D, whose
+    // share starts at ceil(r*D/S); slots are one share apart
+    const uint32_t slot = i_fast ? (uint32_t)((BN + S - 1) / S * C::BM) : (uint32_t)((C::BM + S - 1) / S * C::RED_PITCH);
+    const int own_r = i * S / C::BM;
+    const int row0_r = (own_r * C::BM + S - 1) / S;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t acc[32];
+      if (ok) {
+        tmem_ld32(tmem + lane_addr + c, acc);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0u;
+      }
+      if (i_fast) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = c + e;
+          const int r = j * S / BN;
+          const int j0 = (r * BN + S - 1) / S;
+          const uint32_t off = (rank * slot + (uint32_t)((j - j0) * C::BM + i)) * 4u;
+          st_shared_cluster_f32(mapa_shared(red_base + off, (uint32_t)r), __uint_as_float(acc[e]));
+        }
+      } else {
+        const uint32_t dst =
+            mapa_shared(red_base + (rank * slot + (uint32_t)((i - row0_r) * C::RED_PITCH + c)) * 4u, (uint32_t)own_r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) st_shared_cluster_f32(dst + 4u * e, __uint_as_float(acc[e]));
+      }
+    }
+  }
+
+  // ------------------------------------------------- cluster-wide reduction
+  // After the barrier every slot of this CTA's share holds the partial of
+  // the rank it is named after; sum them in rank order.
+  __syncwarp();                   // reconverge the role warps (the cluster barrier is warp-aligned)
+  tc_fence_before();
+  cluster_sync();
+  {
+    const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
+    const int D = i_fast ? BN : C::BM;                      // the dimension shared out
+    const int inner = i_fast ? C::BM : BN;
+    const int first = (rank * D + S - 1) / S;
+    const int n_own = ((rank + 1) * D + S - 1) / S - first;
+    const int slot = i_fast ? (BN + S - 1) / S * C::BM : (C::BM + S - 1) / S * C::RED_PITCH;
+    const int E = n_own * inner;
+    for (int e = (int)threadIdx.x; e < E; e += C::THREADS) {
+      const int a = e / inner, b = e - a * inner;          // (owned column, row) or (owned row, column)
+      const int i = i_fast ? b : first + a;
+      const int j = i_fast ? first + a : b;
+      const int gi = ta * C::BM + i, gj = tb * BN + j;
+      if (gi >= p.rows_a || gj >= p.rows_b) continue;
+      const int off = i_fast ? a * C::BM + b : a * C::RED_PITCH + b;
+      float acc = red[off];
+#pragma unroll
+      for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
+        if (s2 < S) acc = acc + red[s2 * slot + off];
+      const float v = __fmul_rn(acc, alpha);
+      const int64_t o = (int64_t)gi * p.out_si + (int64_t)gj * p.out_sj;
+      if constexpr (MODE == OUT_BF16) static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(v);
+      else static_cast<float *>(p.out)[o] = v;
+    }
+  }
+  __syncwarp();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace nvfp4

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <utility>
 #include <cstring>
 #include <mutex>
 
@@ -15,6 +16,7 @@
 #include "quantize.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_cluster.cuh"
 
 using namespace nvfp4;
 
@@ -28,6 +30,14 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSplitCluster = 8;
+// CTA-pair GEMM raster: consecutive tiles sweep this many 256-row A tiles
+// before moving to the next B tile column, so that the group's A rows stay
+// in L2 while the B operand streams past them.
+#ifndef NVFP4_PAIR_RASTER_GROUP
+#define NVFP4_PAIR_RASTER_GROUP 8
+#endif
+constexpr int kPairRasterGroup = NVFP4_PAIR_RASTER_GROUP;
 
 std::atomic<uint64_t> g_launches{0};
 std::mutex g_mu;
@@ -37,8 +47,9 @@ struct DeviceState {
   bool ready = false;
   int sms = 0;
   unsigned *err = nullptr;
-  int qtile_bf16 = 1, qtile_f32 = 1;   // resident quantize-tile CTAs per SM
   int pair_clusters = 0;                // co-resident CTA pairs of the pair GEMM
+  // co-resident clusters of the split-K cluster GEMM, [BN 32/64/128][size 1..8]
+  int split_clusters[3][kMaxSplitCluster + 1] = {};
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -56,6 +67,39 @@ cudaError_t set_pair_attrs() {
   cudaError_t e = set_smem(nvfp4_gemm_pair_kernel<OUT_BF16>, b);
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_pair_kernel<OUT_F32>, b);
   return e;
+}
+
+template <int BN>
+cudaError_t set_cluster_attrs() {
+  const int b = ClusterCfg<BN>::SMEM_BYTES;
+  cudaError_t e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, b);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32>, b);
+  return e;
+}
+
+template <typename T>
+cudaError_t set_quant_attrs() {
+  return set_smem(quantize_tma_kernel<T>, QTmaCfg<T>::SMEM_BYTES);
+}
+
+// How many clusters of `size` CTAs of the split-K GEMM fit on the device at once.
+template <int BN>
+int max_split_clusters(int size, int sms) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = size;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(size * sms);
+  cfg.blockDim = dim3(ClusterCfg<BN>::THREADS);
+  cfg.dynamicSmemBytes = ClusterCfg<BN>::SMEM_BYTES;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, &cfg) != cudaSuccess) n = 0;
+  cudaGetLastError();
+  return n;
 }
 
 template <int BN>
@@ -91,8 +135,15 @@ nvfp4_status device_state(DeviceState **out) {
     if (cudaGetSymbolAddress(&errp, g_nvfp4_device_error) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (set_gemm_attrs<256>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
         set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<32>() != cudaSuccess ||
-        set_pair_attrs() != cudaSuccess)
+        set_pair_attrs() != cudaSuccess || set_cluster_attrs<32>() != cudaSuccess ||
+        set_cluster_attrs<64>() != cudaSuccess || set_cluster_attrs<128>() != cudaSuccess ||
+        set_quant_attrs<__nv_bfloat16>() != cudaSuccess || set_quant_attrs<float>() != cudaSuccess)
       return NVFP4_ERR_CUDA;
+    for (int c = 1; c <= kMaxSplitCluster; ++c) {
+      d.split_clusters[0][c] = max_split_clusters<32>(c, sms);
+      d.split_clusters[1][c] = max_split_clusters<64>(c, sms);
+      d.split_clusters[2][c] = max_split_clusters<128>(c, sms);
+    }
     {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -109,13 +160,6 @@ nvfp4_status device_state(DeviceState **out) {
         d.pair_clusters = 0;
       cudaGetLastError();
     }
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qtile_bf16, quantize_tile_kernel<__nv_bfloat16, 4>, 256, 0) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qtile_f32, quantize_tile_kernel<float, 4>, 256, 0) !=
-            cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    if (d.qtile_bf16 < 1) d.qtile_bf16 = 1;
-    if (d.qtile_f32 < 1) d.qtile_f32 = 1;
     d.sms = sms;
     d.err = static_cast<unsigned *>(errp);
     d.ready = true;
@@ -155,35 +199,64 @@ bool make_sf_map(CUtensorMap *map, const void *sf, int64_t rows, int64_t K, int 
   return r == CUDA_SUCCESS;
 }
 
-// GEMM plan: which operand drives the 128-row MMA dimension, the tile width,
-// split-K and the grid.
+// GEMM plan: which kernel, which operand drives the 128-row MMA dimension,
+// the tile width, split-K and the grid.
 struct Plan {
-  bool pair;       // CTA-pair kernel, 256 x 256 tiles
+  enum Kind { SINGLE, PAIR, CLUSTER } kind;
   bool swap;       // A operand = weight (rows N), B operand = activation (rows M)
   int bn;
   int tiles_a, tiles_b, splits, kstages;
   int grid;
 };
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters) {
+inline int narrow_bn(int64_t rows) { return rows <= 32 ? 32 : (rows <= 64 ? 64 : 128); }
+inline int bn_index(int bn) { return bn == 32 ? 0 : (bn == 64 ? 1 : 2); }
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, const DeviceState &d) {
   Plan pl{};
   pl.kstages = (int)((K / 64 + 3) / 4);
-  if (M > 128 && N > 128 && pair_clusters > 0 &&
-      ((M + 255) / 256) * ((N + 255) / 256) >= pair_clusters) {
+  const int sms = d.sms > 0 ? d.sms : 148;
+  if (M > 128 && N > 128 && d.pair_clusters > 0 &&
+      ((M + 255) / 256) * ((N + 255) / 256) >= d.pair_clusters) {
     // large products: CTA pairs on 256 x 256 tiles, one wave of resident pairs
-    pl.pair = true;
+    pl.kind = Plan::PAIR;
     pl.bn = 256;
     pl.tiles_a = (int)((M + 255) / 256);
     pl.tiles_b = (int)((N + 255) / 256);
     pl.splits = 1;
     const int units = pl.tiles_a * pl.tiles_b;
-    pl.grid = 2 * (units < pair_clusters ? units : pair_clusters);
+    pl.grid = 2 * (units < d.pair_clusters ? units : d.pair_clusters);
     return pl;
   }
+  if (M <= 128 || N <= 128) {
+    // one narrow operand: it becomes the MMA's N (decode: the activation;
+    // small-N projections: the weight), the other streams through the
+    // 128-row side, and K is split over the CTAs of a cluster.  The cluster
+    // size minimises waves x (stages per CTA + 1), the +1 standing for the
+    // per-CTA fill and reduction.
+    pl.swap = M <= 128 && (M <= N || N > 128);
+    pl.bn = narrow_bn(pl.swap ? M : N);
+    pl.tiles_a = (int)(((pl.swap ? N : M) + 127) / 128);
+    pl.tiles_b = 1;
+    int best = 0;
+    int64_t best_cost = 0;
+    for (int c = 1; c <= kMaxSplitCluster && c <= pl.kstages; ++c) {
+      const int fit = d.split_clusters[bn_index(pl.bn)][c];
+      if (fit <= 0) continue;
+      const int64_t waves = (pl.tiles_a + fit - 1) / fit;
+      const int64_t cost = waves * ((pl.kstages + c - 1) / c + 1);
+      if (best == 0 || cost < best_cost) { best = c; best_cost = cost; }
+    }
+    if (best > 0) {
+      pl.kind = Plan::CLUSTER;
+      pl.splits = best;
+      pl.grid = pl.tiles_a * best;
+      return pl;
+    }
+  }
+  pl.kind = Plan::SINGLE;
   if (M <= 64) {
-    // decode-shaped: the weight streams through the 128-row MMA dimension and
-    // the few activation rows are the MMA's N; split K so that every SM
-    // (two CTAs each) streams a share of the weight
+    // decode-shaped without cluster support: split-K with a separate reduction
     pl.swap = true;
     pl.bn = M <= 32 ? 32 : 64;
     pl.tiles_a = (int)((N + 127) / 128);
@@ -206,15 +279,48 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters) {
   return pl;
 }
 
-size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters) {
-  const Plan pl = make_plan(M, N, K, sms, pair_clusters);
-  return pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
+size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, const DeviceState &d) {
+  const Plan pl = make_plan(M, N, K, d);
+  return pl.kind == Plan::SINGLE && pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
 }
 
 size_t current_partial_bytes(int64_t M, int64_t N, int64_t K) {
   DeviceState *d = nullptr;
-  if (device_state(&d) != NVFP4_OK) return gemm_partial_bytes(M, N, K, 148, 0);
-  return gemm_partial_bytes(M, N, K, d->sms, d->pair_clusters);
+  if (device_state(&d) != NVFP4_OK) {
+    const DeviceState none{};      // no device: the conservative single-CTA plan
+    return gemm_partial_bytes(M, N, K, none);
+  }
+  return gemm_partial_bytes(M, N, K, *d);
+}
+
+// cudaLaunchKernelEx with an optional cluster shape and programmatic
+// stream serialization (the kernel may start while the preceding one in the
+// stream finishes; it waits for it with griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                      int cluster, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = (unsigned)n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 template <int BN>
@@ -230,20 +336,22 @@ nvfp4_status launch_gemm_bn(const CUtensorMap &ma, const CUtensorMap &mb, const 
   return launched();
 }
 
+// `pdl`: launched right after this library's activation quantize, which
+// lets the GEMM start early and stream the weight while the quantize ends.
 nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
                        const uint8_t *b_codes, const uint8_t *b_sf, const float *b_gscale, void *y,
                        nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K, void *ws,
-                       size_t ws_bytes, cudaStream_t stream) {
+                       size_t ws_bytes, cudaStream_t stream, bool pdl) {
   DeviceState *dev = nullptr;
   nvfp4_status st = device_state(&dev);
   if (st != NVFP4_OK) return st;
   if (M == 0 || N == 0) return NVFP4_OK;
-  const Plan pl = make_plan(M, N, K, dev->sms, dev->pair_clusters);
-  const size_t need = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float) : 0;
+  const Plan pl = make_plan(M, N, K, *dev);
+  const size_t need = gemm_partial_bytes(M, N, K, *dev);
   if (need > 0 && (ws == nullptr || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
   if (need > 0 && !aligned16(ws)) return NVFP4_ERR_ALIGN;
 
-  if (pl.pair) {
+  if (pl.kind == Plan::PAIR) {
     GemmParams p{};
     p.ga = a_gscale;
     p.gb = b_gscale;
@@ -255,7 +363,7 @@ nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float 
     p.tiles_a = pl.tiles_a;
     p.tiles_b = pl.tiles_b;
     p.splits = 1;
-    p.group = 8;
+    p.group = kPairRasterGroup;
     p.err = dev->err;
     p.out = y;
     p.out_si = ld_y;
@@ -279,6 +387,57 @@ nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float 
     cudaError_t e = y_dt == NVFP4_OUT_BF16
                         ? cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_BF16>, ma, mb, msa, msb, p)
                         : cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_F32>, ma, mb, msa, msb, p);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    return launched();
+  }
+
+  if (pl.kind == Plan::CLUSTER) {
+    GemmParams p{};
+    const uint8_t *op_a = pl.swap ? b_codes : a_codes;   // A = 128-row MMA operand
+    const uint8_t *op_b = pl.swap ? a_codes : b_codes;
+    p.sfa = pl.swap ? b_sf : a_sf;
+    p.sfb = pl.swap ? a_sf : b_sf;
+    p.ga = a_gscale;
+    p.gb = b_gscale;
+    p.rows_a = (int)(pl.swap ? N : M);
+    p.rows_b = (int)(pl.swap ? M : N);
+    p.K = (int)K;
+    p.kblocks = (int)(K / 64);
+    p.kstages = pl.kstages;
+    p.tiles_a = pl.tiles_a;
+    p.tiles_b = pl.tiles_b;
+    p.splits = pl.splits;
+    p.group = pl.swap ? 1 : 0;       // which operand is the weight (loaded before the wait)
+    p.err = dev->err;
+    p.out = y;
+    p.out_si = pl.swap ? 1 : ld_y;
+    p.out_sj = pl.swap ? ld_y : 1;
+    CUtensorMap ma, mb;
+    if (!make_codes_map(&ma, op_a, p.rows_a, K, 128) || !make_codes_map(&mb, op_b, p.rows_b, K, pl.bn))
+      return NVFP4_ERR_CUDA;
+    cudaError_t e = cudaSuccess;
+    const bool bf = y_dt == NVFP4_OUT_BF16;
+    const unsigned g = (unsigned)pl.grid;
+    switch (pl.bn) {
+      case 32:
+        e = bf ? launch_ex(nvfp4_gemm_cluster_kernel<32, OUT_BF16>, g, ClusterCfg<32>::THREADS,
+                           ClusterCfg<32>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p)
+               : launch_ex(nvfp4_gemm_cluster_kernel<32, OUT_F32>, g, ClusterCfg<32>::THREADS,
+                           ClusterCfg<32>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p);
+        break;
+      case 64:
+        e = bf ? launch_ex(nvfp4_gemm_cluster_kernel<64, OUT_BF16>, g, ClusterCfg<64>::THREADS,
+                           ClusterCfg<64>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p)
+               : launch_ex(nvfp4_gemm_cluster_kernel<64, OUT_F32>, g, ClusterCfg<64>::THREADS,
+                           ClusterCfg<64>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p);
+        break;
+      default:
+        e = bf ? launch_ex(nvfp4_gemm_cluster_kernel<128, OUT_BF16>, g, ClusterCfg<128>::THREADS,
+                           ClusterCfg<128>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p)
+               : launch_ex(nvfp4_gemm_cluster_kernel<128, OUT_F32>, g, ClusterCfg<128>::THREADS,
+                           ClusterCfg<128>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p);
+        break;
+    }
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     return launched();
   }
@@ -349,25 +508,72 @@ nvfp4_status check_gemm_args(const uint8_t *a_codes, const uint8_t *a_sf, const 
   return NVFP4_OK;
 }
 
+// X viewed as T [rows][K] (row stride ld_x) for the streaming quantize: a
+// box of COLS columns x 128 rows, no swizzle, zeros outside the tensor.
 template <typename T>
-void launch_quantize(const QuantizeParams &p, const DeviceState &dev, cudaStream_t s) {
-  const bool tile_ok = (p.sf_row0 % 128) == 0 && ((p.rows % 128) == 0 || p.pad_rows > 0 || p.rows == 0);
-  if (tile_ok && p.rows > 0) {
-    // one wave of resident CTAs, each looping over 128-row x 512-column tiles
-    const int per_sm = sizeof(T) == 2 ? dev.qtile_bf16 : dev.qtile_f32;
-    const int64_t units = ((p.rows + 127) / 128) * ((p.K + 511) / 512);
-    const int64_t wave = (int64_t)per_sm * dev.sms;
-    const int64_t blocks = units < wave ? units : wave;
-    quantize_tile_kernel<T, 4><<<(unsigned)blocks, 256, 0, s>>>(p);
-    return;
+bool make_x_map(CUtensorMap *map, const void *x, int64_t rows, int64_t K, int64_t ld_x) {
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld_x * (int64_t)sizeof(T))};
+  cuuint32_t box[2] = {(cuuint32_t)QTmaCfg<T>::COLS, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(map, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                        const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename T>
+nvfp4_status launch_quantize(const QuantizeParams &p, const DeviceState &dev, cudaStream_t s, bool pdl) {
+  const bool tile_ok = (p.sf_row0 % 128) == 0 && ((p.rows % 128) == 0 || p.pad_rows > 0);
+  if (tile_ok && p.rows >= 256) {
+    // streaming kernel: one CTA per SM over 128-row units
+    CUtensorMap mx;
+    if (!make_x_map<T>(&mx, p.x, p.rows, p.K, p.ld_x)) return NVFP4_ERR_CUDA;
+    using C = QTmaCfg<T>;
+    const int64_t units = ((p.rows + 127) / 128) * ((p.K + C::COLS - 1) / C::COLS);
+    const unsigned grid = (unsigned)(units < dev.sms ? units : dev.sms);
+    if (launch_ex(quantize_tma_kernel<T>, grid, C::THREADS, C::SMEM_BYTES, s, 0, pdl, mx, p) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    return launched();
   }
-  constexpr int U = 4;
-  const int64_t nseg = (p.K + 255) / 256;
-  const int64_t units = p.rows * nseg;
-  int64_t blocks = ((units + U - 1) / U + 7) / 8;
-  if (blocks > 8LL * dev.sms) blocks = 8LL * dev.sms;
-  if (blocks < 1) blocks = 1;
-  quantize_kernel<T, U><<<(unsigned)blocks, 256, 0, s>>>(p);
+  // generic kernel: one warp per 512-column row segment; few rows (decode)
+  // get one segment per warp so that the kernel is as short as possible
+  const int64_t units = p.rows * ((p.K + 511) / 512);
+  cudaError_t e;
+  if (units >= 32LL * dev.sms) {
+    int64_t blocks = (units / 4 + 7) / 8;
+    if (blocks > 8LL * dev.sms) blocks = 8LL * dev.sms;
+    e = launch_ex(quantize_rows_kernel<T, 4>, (unsigned)blocks, 256u, 0, s, 0, pdl, p);
+  } else {
+    int64_t blocks = (units + 7) / 8;
+    if (blocks < 1) blocks = 1;
+    e = launch_ex(quantize_rows_kernel<T, 1>, (unsigned)blocks, 256u, 0, s, 0, pdl, p);
+  }
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return launched();
+}
+
+nvfp4_status quantize_impl(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                           const float *gscale, uint8_t *codes, uint8_t *sf, int64_t sf_row0, int64_t sf_rows_total,
+                           cudaStream_t s, bool pdl) {
+  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || sf_row0 < 0 || sf_rows_total < sf_row0 + rows ||
+      rows * ((K + 255) / 256) >= (int64_t)UINT32_MAX)
+    return NVFP4_ERR_SHAPE;
+  const bool owns_pad = sf_row0 + rows == sf_rows_total;
+  const int64_t pad_rows = owns_pad ? pad128(sf_rows_total) - sf_rows_total : 0;
+  if (rows == 0 && pad_rows == 0) return NVFP4_OK;
+  if (!sf || !gscale || (rows > 0 && (!x || !codes))) return NVFP4_ERR_NULL;
+  const int esz = dt == NVFP4_IN_BF16 ? 2 : 4;
+  if ((rows > 0 && (!aligned16(x) || !aligned16(codes))) || (ld_x * esz) % 16 != 0 || !aligned16(sf))
+    return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  QuantizeParams p{x, rows, K, ld_x, gscale, codes, sf, sf_row0, pad_rows, dev->err};
+  return dt == NVFP4_IN_BF16 ? launch_quantize<__nv_bfloat16>(p, *dev, s, pdl)
+                             : launch_quantize<float>(p, *dev, s, pdl);
 }
 
 }  // namespace
@@ -416,24 +622,8 @@ nvfp4_status nvfp4_amax_gscale(const void *x, nvfp4_in_dtype dt, int64_t rows, i
 nvfp4_status nvfp4_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
                             const float *gscale, uint8_t *codes, uint8_t *sf, int64_t sf_row0,
                             int64_t sf_rows_total, nvfp4_stream_t stream) {
-  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
-  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || sf_row0 < 0 || sf_rows_total < sf_row0 + rows ||
-      rows * ((K + 255) / 256) >= (int64_t)UINT32_MAX)
-    return NVFP4_ERR_SHAPE;
-  const bool owns_pad = sf_row0 + rows == sf_rows_total;
-  const int64_t pad_rows = owns_pad ? pad128(sf_rows_total) - sf_rows_total : 0;
-  if (rows == 0 && pad_rows == 0) return NVFP4_OK;
-  if (!sf || !gscale || (rows > 0 && (!x || !codes))) return NVFP4_ERR_NULL;
-  const int esz = dt == NVFP4_IN_BF16 ? 2 : 4;
-  if ((rows > 0 && (!aligned16(x) || !aligned16(codes))) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
-  DeviceState *dev = nullptr;
-  nvfp4_status st = device_state(&dev);
-  if (st != NVFP4_OK) return st;
-  QuantizeParams p{x, rows, K, ld_x, gscale, codes, sf, sf_row0, pad_rows};
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dt == NVFP4_IN_BF16) launch_quantize<__nv_bfloat16>(p, *dev, s);
-  else launch_quantize<float>(p, *dev, s);
-  return launched();
+  return quantize_impl(x, dt, rows, K, ld_x, gscale, codes, sf, sf_row0, sf_rows_total,
+                       reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 nvfp4_status nvfp4_harmonize_group(uint8_t *sf, int64_t rows_total, int64_t K, int n_modules,
@@ -477,7 +667,7 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float
   nvfp4_status st = check_gemm_args(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, y, y_dt, ld_y, M, N, K);
   if (st != NVFP4_OK || M == 0 || N == 0) return st;
   return gemm_impl(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, y, y_dt, ld_y, M, N, K, workspace,
-                   workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+                   workspace_bytes, reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -507,12 +697,12 @@ nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const f
   if (st != NVFP4_OK) return st;
   DeviceState *dev = nullptr;
   if ((st = device_state(&dev)) != NVFP4_OK) return st;
-  if (workspace_bytes < codes_b + sf_b + gemm_partial_bytes(M, N, K, dev->sms, dev->pair_clusters))
-    return NVFP4_ERR_WORKSPACE;
-  st = nvfp4_quantize(x, x_dt, M, K, ld_x, x_gscale, a_codes, a_sf, 0, M, stream);
+  if (workspace_bytes < codes_b + sf_b + gemm_partial_bytes(M, N, K, *dev)) return NVFP4_ERR_WORKSPACE;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = quantize_impl(x, x_dt, M, K, ld_x, x_gscale, a_codes, a_sf, 0, M, s, true);
   if (st != NVFP4_OK) return st;
-  return gemm_impl(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K,
-                   a_sf + sf_b, workspace_bytes - codes_b - sf_b, reinterpret_cast<cudaStream_t>(stream));
+  return gemm_impl(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K, a_sf + sf_b,
+                   workspace_bytes - codes_b - sf_b, s, true);
 }
 
 nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,

@@ -297,4 +297,25 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t mask) {
       "h"(mask)
       : "memory");
 }
+// ------------------------------------------- programmatic dependent launch
+// Block until the grids this one depends on (launched earlier in the stream
+// with programmatic serialization) have completed and their writes are
+// visible; a no-op for a grid launched without that attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next grid in the stream be scheduled (it still waits for this grid
+// where it executes griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// store a float into the shared memory of a CTA of this cluster (the
+// address from mapa); ordered before a later barrier.cluster.arrive.release
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t cluster_addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+// read a float from the shared memory of a CTA of this cluster
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
 }  // namespace nvfp4

@@ -10,6 +10,7 @@
 // with round-to-nearest-even and saturation at 448 / 6; a block whose scale
 // or d is zero gets +0 codes.
 #pragma once
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -23,88 +24,102 @@ __device__ __forceinline__ int64_t sf_index(int64_t r, int64_t c, int64_t K) {
   return ((r >> 7) * (K >> 6) + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
 }
 
+// ------------------------------------------------------------ input blocks
+// One 16-element scale block of the input as loaded: bf16 as eight packed
+// pairs (element 2i in the low half of word i), fp32 as sixteen floats.
 template <typename T>
-struct Vec8;  // eight consecutive input elements as fp32
+struct Block16;
 
 template <>
-struct Vec8<__nv_bfloat16> {
-  uint4 raw;
-  __device__ __forceinline__ void zero() { raw = make_uint4(0u, 0u, 0u, 0u); }
-  __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
-    raw = __ldg(reinterpret_cast<const uint4 *>(p));
-  }
-  __device__ __forceinline__ void to_f32(float (&v)[8]) const {
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-};
-
-template <>
-struct Vec8<float> {
-  float4 a, b;
-  __device__ __forceinline__ void zero() {
-    a = make_float4(0.f, 0.f, 0.f, 0.f);
-    b = a;
-  }
-  __device__ __forceinline__ void load(const float *p) {
-    a = __ldg(reinterpret_cast<const float4 *>(p));
-    b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-  }
-  __device__ __forceinline__ void to_f32(float (&v)[8]) const {
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
-};
-
-template <typename T>
-struct Vec16;  // sixteen consecutive input elements (one scale block)
-
-template <>
-struct Vec16<__nv_bfloat16> {
-  uint4 a, b;
-  __device__ __forceinline__ void zero() { a = b = make_uint4(0u, 0u, 0u, 0u); }
-  __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
-    a = __ldg(reinterpret_cast<const uint4 *>(p));
-    b = __ldg(reinterpret_cast<const uint4 *>(p) + 1);
-  }
-  __device__ __forceinline__ void to_f32(float (&v)[16]) const {
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-};
-
-template <>
-struct Vec16<float> {
-  float4 q[4];
+struct Block16<__nv_bfloat16> {
+  uint32_t w[8];
   __device__ __forceinline__ void zero() {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < 8; ++i) w[i] = 0u;
+  }
+  __device__ __forceinline__ void set(uint4 a, uint4 b) {
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+    set(__ldg(reinterpret_cast<const uint4 *>(p)), __ldg(reinterpret_cast<const uint4 *>(p) + 1));
+  }
+  __device__ __forceinline__ void load_shared(const __nv_bfloat16 *p) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+    set(q[0], q[1]);
+  }
+  __device__ __forceinline__ float elem(int e) const {      // e a compile-time index
+    return __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+  }
+  // max |x| of the block: a tree of bf16x2 max-of-magnitudes, then the two halves
+  __device__ __forceinline__ float amax() const {
+    uint32_t a = bmax2(bmax2(bmax2(w[0], w[1]), bmax2(w[2], w[3])), bmax2(bmax2(w[4], w[5]), bmax2(w[6], w[7])));
+    a &= 0x7FFF7FFFu;
+    return fmaxf(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+  }
+  static __device__ __forceinline__ uint32_t bmax2(uint32_t x, uint32_t y) {
+    uint32_t m;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(x), "r"(y));
+    return m;
+  }
+};
+
+template <>
+struct Block16<float> {
+  float v[16];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+  }
+  __device__ __forceinline__ void set4(int i, float4 a) {
+    v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
   }
   __device__ __forceinline__ void load(const float *p) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = __ldg(reinterpret_cast<const float4 *>(p) + i);
+    for (int i = 0; i < 4; ++i) set4(i, __ldg(reinterpret_cast<const float4 *>(p) + i));
   }
-  __device__ __forceinline__ void to_f32(float (&v)[16]) const {
+  __device__ __forceinline__ void load_shared(const float *p) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[4 * i] = q[i].x; v[4 * i + 1] = q[i].y; v[4 * i + 2] = q[i].z; v[4 * i + 3] = q[i].w;
-    }
+    for (int i = 0; i < 4; ++i) set4(i, reinterpret_cast<const float4 *>(p)[i]);
+  }
+  __device__ __forceinline__ float elem(int e) const { return v[e]; }
+  __device__ __forceinline__ float amax() const {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    return m;
   }
 };
 
-// Per-tensor constants of the encoder.
+__device__ __forceinline__ float to_f32(__nv_bfloat16 h) { return __bfloat162float(h); }
+__device__ __forceinline__ float to_f32(float f) { return f; }
+
+// --------------------------------------------------------------- the encoder
+// The definition (each step one IEEE fp32 operation, round to nearest even):
+//   s = E4M3(fl32(amax / fl32(6g))),  d = fl32(dec(s) * g),  q_i = E2M1(fl32(x_i / d)).
+// The encoder reaches the same codes without a division.  With
+// r = fl32(fl32(1/dec(s)) * fl32(1/g)) (relative error <= 3u, u = 2^-24), the
+// products y- = fl32(x * fl32(r(1 - 2^-21))) and y+ = fl32(x * fl32(r(1 + 2^-21)))
+// bracket the exact quotient fl32(x/d) in magnitude (margin >= u after all
+// roundings), and E2M1 rounding is monotone in |y|: where the hardware
+// conversion gives the same code for y- and y+, that is the code of
+// fl32(x/d).  Where the two codes differ (the bracket is far narrower than the
+// grid, so they are neighbours and the bracket holds exactly one rounding
+// boundary T, one of 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5), the side of T on
+// which fl32(x/d) falls is decided exactly (see quotient_vs).  The scale
+// byte is decided the same way from amax * fl32(1/g6) widened by 2^-21 both
+// ways, with the midpoint between the two candidate E4M3 values as T.  With
+// bf16 inputs, quotients land on or next to a boundary for a few elements
+// in a thousand (exact ties included), so this path must stay cheap.
+constexpr float kWidenLo = 0.999999523162841796875f;   // 1 - 2^-21
+constexpr float kWidenHi = 1.000000476837158203125f;   // 1 + 2^-21
+
+// rounding boundary between E2M1 magnitudes m and m + 1
+__constant__ float kE2m1Boundary[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+
 struct EncodeConsts {
-  float g, g6;      // global scale and fl32(6*g)
-  float rg, rg6;    // fl32(1/g), fl32(1/g6)
-  bool fast;        // the multiply-by-reciprocal path is usable (g well inside the normal range)
+  float g, g6, rg;          // g, fl32(6g), fl32(1/g)
+  float rg6_lo, rg6_hi;     // fl32(1/g6) widened down and up by 2^-21
+  bool fast;                // g well inside the normal range: products neither overflow nor underflow
 };
 
 __device__ __forceinline__ EncodeConsts encode_consts(const float *gscale) {
@@ -112,7 +127,9 @@ __device__ __forceinline__ EncodeConsts encode_consts(const float *gscale) {
   k.g = __ldg(gscale);
   k.g6 = __fmul_rn(6.0f, k.g);
   k.rg = __frcp_rn(k.g);
-  k.rg6 = __frcp_rn(k.g6);
+  const float rg6 = __frcp_rn(k.g6);
+  k.rg6_lo = __fmul_rn(rg6, kWidenLo);
+  k.rg6_hi = __fmul_rn(rg6, kWidenHi);
   k.fast = k.g >= 8.67361738e-19f && k.g <= 1.15292150e18f;   // 2^-60 .. 2^60
   return k;
 }
@@ -124,93 +141,128 @@ __device__ __forceinline__ void fill_rcp_table(float *tab) {
     tab[i] = i == 0 || i == 127 ? 0.0f : __frcp_rn(e4m3_to_f32((uint32_t)i));
 }
 
-// IEEE reference path of one half-block: t = amax / g6, y = x / (dec(s)*g).
-__device__ __noinline__ uint32_t encode8_ieee(const float *v, float amax, float g, float g6, uint32_t *s_out) {
-  const uint32_t s = f32_to_e4m3(__fdiv_rn(amax, g6));
-  *s_out = s;
-  const float d = __fmul_rn(e4m3_to_f32(s), g);
-  if (s == 0u || d == 0.0f) return 0u;
-  float y[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(v[i], d);
-  return f32x8_to_e2m1(y);
-}
-
-// Encode eight values of one half-block given the block's amax; returns the
-// packed code word and (through *s_out) the E4M3 scale byte.  The result is
-// bit-identical to the IEEE definition
-//   s = E4M3(fl32(amax / fl32(6g))),  q_i = E2M1(fl32(x_i / fl32(dec(s) g))).
-// Fast path: t' = fl32(amax * fl32(1/g6)) is within 2 ulps of fl32(amax/g6)
-// and y' = fl32(fl32(x * fl32(1/dec(s))) * fl32(1/g)) within 6 ulps of
-// fl32(x/d).  A rounding decision can only differ if a decision point lies
-// between the two values: every E4M3 midpoint has 19 and every E2M1 decision
-// threshold (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) 21 trailing zero bits in its
-// fp32 encoding, so a value whose bit pattern is not within 8 of such a
-// multiple is decided exactly.  Otherwise (and for extreme g) the IEEE path
-// recomputes the group.
-__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float amax, const EncodeConsts &k,
-                                            const float *rcp_tab, uint32_t *s_out) {
-  if (!k.fast) return encode8_ieee(v, amax, k.g, k.g6, s_out);
-  const float t = __fmul_rn(amax, k.rg6);
-  if (((__float_as_uint(t) + 8u) & 0x7FFF0u) == 0u) return encode8_ieee(v, amax, k.g, k.g6, s_out);
-  const uint32_t s = f32_to_e4m3(t);
-  *s_out = s;
-  if (s == 0u) return 0u;
-  const float rs = rcp_tab[s];
-  float y[8];
-  uint32_t near = 0xFFFFFFFFu;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    y[i] = __fmul_rn(__fmul_rn(v[i], rs), k.rg);
-    const uint32_t b = __float_as_uint(y[i]) & 0x7FFFFFFFu;
-    near = min(near, ((b + 8u) & 0x1FFFF0u) | (b < 0x3E000000u ? 1u : 0u));
-  }
-  if (near == 0u) return encode8_ieee(v, amax, k.g, k.g6, s_out);
-  return f32x8_to_e2m1(y);
-}
-
 __device__ __noinline__ float div_rn_slow(float a, float b) { return __fdiv_rn(a, b); }
 
-// One whole 16-element block.  Same definition and exactness argument as
-// encode8, applied per value: t' = fl32(amax * fl32(1/g6)) and
-// y' = fl32(x * fl32(fl32(1/dec(s)) * fl32(1/g))) are within 2 and 6 ulps of
-// the IEEE results; only a value whose bit pattern lies within 8 of a multiple
-// of 2^19 (t) or 2^21 (y) -- a superset of the decision points -- is
-// recomputed with IEEE division, one value at a time.  (With bf16 inputs and
-// block scales built from them, values land next to round numbers far more
-// often than chance, so recomputing whole blocks would be costly.)
-__device__ __forceinline__ uint2 encode16(const float (&v)[16], float amax, const EncodeConsts &k,
-                                          const float *rcp_tab, uint32_t *s_out) {
-  float t = __fmul_rn(amax, k.rg6);
-  if (!k.fast || ((__float_as_uint(t) + 8u) & 0x7FFF0u) == 0u) t = div_rn_slow(amax, k.g6);
-  const uint32_t s = f32_to_e4m3(t);
+// Sign of fl32(a / b) - T for a >= 0 and b > 0 normal, T > 0 a normal float
+// with a short significand (an E2M1 boundary or an E4M3 midpoint).  With h+
+// and h- half the float spacing above and below T, RNE gives fl32(a/b) > T
+// exactly when a/b > T + h+, and fl32(a/b) < T exactly when a/b < T - h-
+// (at either bound the tie goes to T, whose last significand bit is 0).
+// Compared as a vs (T +- h) * b in fp64: T +- h needs at most 26 significant
+// bits and b 24, so the product and the comparison are exact.
+__device__ __forceinline__ int quotient_vs(float a, float b, float T) {
+  const uint32_t tb = __float_as_uint(T);
+  const long long e = (long long)((tb >> 23) & 0xFFu) - 127 - 24 + 1023;   // exponent of h+ = ulp(T)/2
+  const double hp = __longlong_as_double(e << 52);
+  const double hm = (tb & 0x7FFFFFu) == 0u ? 0.5 * hp : hp;    // below a power of two the spacing halves
+  const double da = (double)a, db = (double)b, dt = (double)T;
+  if (da > __dmul_rn(dt + hp, db)) return 1;
+  if (da < __dmul_rn(dt - hm, db)) return -1;
+  return 0;
+}
+
+// E2M1 codes of eight values under the two bracketing multipliers: the code
+// word from r- and the code word from r+ (element 2j in the low nibble of byte j).
+__device__ __forceinline__ void e2m1x8_bracket(float x0, float x1, float x2, float x3, float x4, float x5,
+                                               float x6, float x7, float rlo, float rhi, uint32_t &wlo,
+                                               uint32_t &whi) {
+  asm("{\n\t"
+      ".reg .b64 a0, a1, a2, a3, bl, bh, d;\n\t"
+      ".reg .f32 p0, p1;\n\t"
+      ".reg .b8 l0, l1, l2, l3, h0, h1, h2, h3;\n\t"
+      "mov.b64 bl, {%10, %10};\n\t"
+      "mov.b64 bh, {%11, %11};\n\t"
+      "mov.b64 a0, {%2, %3};\n\t"
+      "mov.b64 a1, {%4, %5};\n\t"
+      "mov.b64 a2, {%6, %7};\n\t"
+      "mov.b64 a3, {%8, %9};\n\t"
+      "mul.rn.f32x2 d, a0, bl;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 l0, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a1, bl;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 l1, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a2, bl;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 l2, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a3, bl;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 l3, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a0, bh;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 h0, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a1, bh;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 h1, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a2, bh;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 h2, p1, p0;\n\t"
+      "mul.rn.f32x2 d, a3, bh;\n\t mov.b64 {p0, p1}, d;\n\t cvt.rn.satfinite.e2m1x2.f32 h3, p1, p0;\n\t"
+      "mov.b32 %0, {l0, l1, l2, l3};\n\t"
+      "mov.b32 %1, {h0, h1, h2, h3};\n\t"
+      "}"
+      : "=r"(wlo), "=r"(whi)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7), "f"(rlo), "f"(rhi));
+}
+
+// E2M1 code (nibble) of one value, satfinite, round to nearest even.
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  uint16_t b;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %1, %1;\n\tcvt.u16.u8 %0, c;\n\t}" : "=h"(b) : "f"(y));
+  return b & 0xFu;
+}
+
+// Settle the elements whose bracket codes differ (nonzero nibbles of
+// lo ^ hi): the lower candidate magnitude m fixes the boundary T between m
+// and m + 1; the element takes m + 1 above T, m below, the even one of the
+// two on T.  `src` is the block in memory (elements re-read by index).
+template <typename T>
+__device__ __forceinline__ uint2 settle_codes(const T *src, uint64_t lo, uint64_t hi, float d) {
+  uint64_t m = lo ^ hi;
+  while (m != 0ull) {
+    const int sh = (__ffsll((long long)m) - 1) & ~3;
+    m &= ~(0xFull << sh);
+    const uint32_t cl = (uint32_t)(lo >> sh) & 7u, ch = (uint32_t)(hi >> sh) & 7u;
+    const uint32_t mlow = min(cl, ch);
+    const float xv = to_f32(src[sh >> 2]);
+    const int c = quotient_vs(fabsf(xv), d, kE2m1Boundary[mlow]);
+    const uint32_t mag = c > 0 ? mlow + 1u : (c < 0 ? mlow : ((mlow & 1u) ? mlow + 1u : mlow));
+    const uint32_t code = mag | ((__float_as_uint(xv) >> 28) & 8u);
+    lo = (lo & ~(0xFull << sh)) | ((uint64_t)code << sh);
+  }
+  return make_uint2((uint32_t)lo, (uint32_t)(lo >> 32));
+}
+
+// The whole block by the definition (extreme global scales only).
+template <typename T>
+__device__ __noinline__ uint2 encode16_ieee(const T *src, uint32_t s, float g) {
+  const float d = __fmul_rn(e4m3_to_f32(s), g);
+  if (d == 0.0f) return make_uint2(0u, 0u);
+  uint32_t w[2] = {0u, 0u};
+  for (int e = 0; e < 16; ++e) w[e >> 3] |= e2m1_code(__fdiv_rn(to_f32(src[e]), d)) << ((e & 7) * 4);
+  return make_uint2(w[0], w[1]);
+}
+
+// Encode one 16-element block held in registers (`src` is the same block in
+// memory, read only on the rare settling paths).  Returns the two code
+// words; the scale byte goes to *s_out.
+template <typename T>
+__device__ __forceinline__ uint2 encode16(const Block16<T> &b, const EncodeConsts &k, const float *rcp_tab,
+                                          const T *src, uint32_t *s_out) {
+  const float amax = b.amax();
+  uint16_t pr;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(__fmul_rn(amax, k.rg6_hi)),
+      "f"(__fmul_rn(amax, k.rg6_lo)));
+  uint32_t s = pr & 0xFFu;
+  const uint32_t s_up = (uint32_t)(pr >> 8);
+  if (!k.fast) {
+    s = f32_to_e4m3(div_rn_slow(amax, k.g6));
+  } else if (s != s_up) {
+    // neighbouring E4M3 values: decide against their midpoint
+    const float mid = __fmul_rn(__fadd_rn(e4m3_to_f32(s), e4m3_to_f32(s_up)), 0.5f);
+    const int c = quotient_vs(amax, k.g6, mid);
+    s = c > 0 ? s_up : (c < 0 ? s : ((s & 1u) ? s_up : s));
+  }
   *s_out = s;
   if (s == 0u) return make_uint2(0u, 0u);
-  float y[16];
-  if (k.fast) {
-    const float r = __fmul_rn(rcp_tab[s], k.rg);
-    uint32_t near = 0xFFFFFFFFu;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      y[i] = __fmul_rn(v[i], r);
-      near = min(near, (__float_as_uint(y[i]) + 8u) & 0x1FFFF0u);
-    }
-    if (near == 0u) {
-      const float d = __fmul_rn(e4m3_to_f32(s), k.g);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (((__float_as_uint(y[i]) + 8u) & 0x1FFFF0u) == 0u) y[i] = div_rn_slow(v[i], d);
-    }
-  } else {
-    const float d = __fmul_rn(e4m3_to_f32(s), k.g);
-    if (d == 0.0f) return make_uint2(0u, 0u);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = div_rn_slow(v[i], d);
-  }
-  uint2 out;
-  out.x = f32x8_to_e2m1(*reinterpret_cast<const float(*)[8]>(&y[0]));
-  out.y = f32x8_to_e2m1(*reinterpret_cast<const float(*)[8]>(&y[8]));
-  return out;
+  if (!k.fast) return encode16_ieee(src, s, k.g);
+  const float r = __fmul_rn(rcp_tab[s], k.rg);
+  const float rlo = __fmul_rn(r, kWidenLo), rhi = __fmul_rn(r, kWidenHi);
+  uint32_t lo0, hi0, lo1, hi1;
+  e2m1x8_bracket(b.elem(0), b.elem(1), b.elem(2), b.elem(3), b.elem(4), b.elem(5), b.elem(6), b.elem(7), rlo, rhi,
+                 lo0, hi0);
+  e2m1x8_bracket(b.elem(8), b.elem(9), b.elem(10), b.elem(11), b.elem(12), b.elem(13), b.elem(14), b.elem(15), rlo,
+                 rhi, lo1, hi1);
+  if (((lo0 ^ hi0) | (lo1 ^ hi1)) != 0u)
+    return settle_codes(src, (uint64_t)lo0 | ((uint64_t)lo1 << 32), (uint64_t)hi0 | ((uint64_t)hi1 << 32),
+                        __fmul_rn(e4m3_to_f32(s), k.g));
+  return make_uint2(lo0, lo1);
 }
 
 struct QuantizeParams {
@@ -221,54 +273,56 @@ struct QuantizeParams {
   uint8_t *sf;
   int64_t sf_row0;
   int64_t pad_rows;  // padding rows (zeroed) after this call's rows, or 0
+  unsigned *err;
 };
 
-// Generic path (any row offset inside a fused buffer): one warp handles a
-// 256-element segment of one row per unit; lane l owns elements [8l, 8l+8),
-// lanes 2i and 2i+1 form 16-element block i and exchange their half-maxima
-// with one shuffle.  Loads are 16-byte vectors, code words 4-byte stores, and
-// every scale byte is stored on its own.  UNROLL units are loaded before any
-// is encoded.
+// Programmatic-dependent-launch prologue of every kernel that reads what an
+// earlier kernel wrote: wait for the stream's preceding grid, then let the
+// next one be scheduled (it in turn waits for this grid where it must).
+__device__ __forceinline__ void pdl_prologue() {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+}
+
+// Generic path (any row offset inside a fused buffer, any row count): one
+// warp per 512-column segment of a row, lane l encodes block l of it (32
+// bytes of bf16 per lane, 1 KB contiguous per warp), UNROLL segments loaded
+// before any is encoded.  Codes are 8-byte stores, each scale byte is stored
+// on its own.
 template <typename T, int UNROLL>
-__global__ void __launch_bounds__(256) quantize_kernel(QuantizeParams p) {
+__global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
+  __shared__ float rcp_tab[128];
+  fill_rcp_table(rcp_tab);
+  pdl_prologue();
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  const uint32_t nseg = (uint32_t)((p.K + 255) >> 8);
+  const uint32_t nseg = (uint32_t)((p.K + 511) >> 9);
   const uint32_t units = (uint32_t)p.rows * nseg;
   const int64_t ncols = p.K >> 4;
-  __shared__ float rcp_tab[128];
-  fill_rcp_table(rcp_tab);
-  __syncthreads();
   const EncodeConsts kc = encode_consts(p.gscale);
   const T *x = static_cast<const T *>(p.x);
 
   for (uint32_t u0 = warp * UNROLL; u0 < units; u0 += nwarps * UNROLL) {
-    Vec8<T> in[UNROLL];
+    Block16<T> in[UNROLL];
     int64_t row[UNROLL];
     int col[UNROLL];
 #pragma unroll
     for (int j = 0; j < UNROLL; ++j) {
       const uint32_t u = u0 + j;
       row[j] = u / nseg;
-      col[j] = (int)(u - (uint32_t)row[j] * nseg) * 256 + lane * 8;
+      col[j] = (int)(u - (uint32_t)row[j] * nseg) * 512 + lane * 16;
       in[j].zero();
       if (u < units && col[j] < p.K) in[j].load(x + row[j] * p.ld_x + col[j]);
     }
 #pragma unroll
     for (int j = 0; j < UNROLL; ++j) {
-      const bool active = u0 + j < units && col[j] < p.K;
-      float v[8];
-      in[j].to_f32(v);
-      float amax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-      if (active) {
+      if (u0 + j < units && col[j] < p.K) {
         uint32_t s;
-        const uint32_t word = encode8(v, amax, kc, rcp_tab, &s);
-        *reinterpret_cast<uint32_t *>(p.codes + row[j] * (p.K >> 1) + (col[j] >> 1)) = word;
-        if ((lane & 1) == 0) p.sf[sf_index(p.sf_row0 + row[j], col[j] >> 4, p.K)] = static_cast<uint8_t>(s);
+        const uint2 word = encode16(in[j], kc, rcp_tab, x + row[j] * p.ld_x + col[j], &s);
+        *reinterpret_cast<uint2 *>(p.codes + row[j] * (p.K >> 1) + (col[j] >> 1)) = word;
+        p.sf[sf_index(p.sf_row0 + row[j], col[j] >> 4, p.K)] = static_cast<uint8_t>(s);
       }
     }
   }
@@ -282,66 +336,121 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantizeParams p) {
   }
 }
 
-// Tile path, used when this call's scale rows start on a 128-row boundary and
-// it owns every row of its last 128-row block (the activation quantize always
-// does).  A CTA of 8 warps handles a 128-row x 512-column tile; lane l of a
-// warp encodes 16-element block l of a row segment (32 contiguous bytes of
-// bf16 per lane, 1 KB per warp-row), warp w takes rows w, w+8, ..., w+120.
-// The tile's 32 scale columns -- exactly eight 512-byte atoms, contiguous in
-// the swizzled buffer -- are collected in shared memory and written with
-// 16-byte stores.  Rows past `rows` (padding) get zero scales.
-template <typename T, int UNROLL>
-__global__ void __launch_bounds__(256) quantize_tile_kernel(QuantizeParams p) {
-  __shared__ __align__(16) uint8_t sf_tile[4096];
-  __shared__ float rcp_tab[128];
-  fill_rcp_table(rcp_tab);
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t nseg = (uint32_t)((p.K + 511) >> 9);
-  const uint32_t nrb = (uint32_t)((p.rows + 127) >> 7);
-  const uint32_t units = nrb * nseg;
-  const uint32_t atoms_per_rb = (uint32_t)(p.K >> 6);
-  const EncodeConsts kc = encode_consts(p.gscale);
-  const T *x = static_cast<const T *>(p.x);
-  const int sf_off = (lane >> 2) * 512 + (lane & 3);     // this lane's block column inside the tile
+// Streaming path for calls whose scale rows start on a 128-row boundary and
+// that own every row of their last 128-row block (the activation quantize
+// always does).  One CTA per SM, persistent over units of 128 rows x COLS
+// columns (64 KB of input; COLS = 256 bf16 / 128 fp32):
+//   warp 0       one thread streams units into a ring of shared-memory stages
+//                with 2D TMA loads (rows past `rows` and columns past K read
+//                as zeros, so padding rows get zero scales);
+//   warps 1..16  encode: lane l takes block l % (COLS/16) of row
+//                l / (COLS/16) of each step and writes its 8 code bytes and
+//                its scale byte straight to global memory (a warp's scale
+//                bytes fill 4-byte runs of the swizzled atoms, which the L2
+//                merges); each warp hands the stage back on its own, so the
+//                warps never wait for one another.
+template <typename T>
+struct QTmaCfg {
+  static constexpr int ROWS = 128;
+  static constexpr int COLS = sizeof(T) == 2 ? 256 : 128;
+  static constexpr int BPR = COLS / 16;                 // blocks per row
+  static constexpr int RPS = 32 / BPR;                  // rows per warp step
+  static constexpr int CONSUMERS = 16;
+  static constexpr int SPW = ROWS / RPS / CONSUMERS;    // steps per warp per unit
+  static constexpr int STAGE_BYTES = ROWS * COLS * (int)sizeof(T);
+  static constexpr int STAGES = 3;
+  static constexpr int THREADS = 32 * (1 + CONSUMERS);
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * STAGES * 8 + 512 + 16;
+  static_assert(ROWS % (RPS * CONSUMERS) == 0, "unit split");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
 
-  for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
-    const uint32_t rb = u / nseg, seg = u - rb * nseg;
-    const int col = (int)seg * 512 + lane * 16;
-    const bool col_ok = col < p.K;
-    const int64_t row0 = (int64_t)rb * 128 + warp;
-    const T *xp = x + row0 * p.ld_x + col;
-    uint8_t *cp = p.codes + row0 * (p.K >> 1) + (col >> 1);
-#pragma unroll 1
-    for (int i0 = 0; i0 < 16; i0 += UNROLL) {
-      Vec16<T> in[UNROLL];
-#pragma unroll
-      for (int j = 0; j < UNROLL; ++j) {
-        in[j].zero();
-        if (col_ok && row0 + 8 * (i0 + j) < p.rows) in[j].load(xp + (int64_t)(8 * (i0 + j)) * p.ld_x);
-      }
-#pragma unroll
-      for (int j = 0; j < UNROLL; ++j) {
-        const int rl = warp + 8 * (i0 + j);
-        float v[16];
-        in[j].to_f32(v);
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        uint32_t s = 0;
-        if (col_ok && row0 + 8 * (i0 + j) < p.rows) {
-          const uint2 word = encode16(v, amax, kc, rcp_tab, &s);
-          *reinterpret_cast<uint2 *>(cp + (int64_t)(8 * (i0 + j)) * (p.K >> 1)) = word;
-        }
-        sf_tile[sf_off + (rl & 31) * 16 + (rl >> 5) * 4] = (uint8_t)s;
+template <typename T>
+__global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
+    quantize_tma_kernel(const __grid_constant__ CUtensorMap tmx, const QuantizeParams p) {
+  using C = QTmaCfg<T>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *ring = smem;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + C::STAGES * C::STAGE_BYTES);
+  uint64_t *empty = full + C::STAGES;
+  float *rcp_tab = reinterpret_cast<float *>(empty + C::STAGES);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(rcp_tab + 128);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t nseg = (uint32_t)((p.K + C::COLS - 1) / C::COLS);
+  const uint32_t units = (uint32_t)((p.rows + 127) >> 7) * nseg;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::CONSUMERS);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmx);
+  }
+  fill_rcp_table(rcp_tab);
+  pdl_prologue();
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int st = 0;
+      uint32_t ph = 0;
+      for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
+        if (!mbar_wait(&empty[st], ph ^ 1, p.err, ERR_PRODUCER, abort_flag)) break;
+        const uint32_t rb = u / nseg, seg = u - rb * nseg;
+        mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+        tma_load_2d(ring + st * C::STAGE_BYTES, &tmx, &full[st], (int32_t)(seg * C::COLS), (int32_t)(rb * 128));
+        if (++st == C::STAGES) { st = 0; ph ^= 1; }
       }
     }
-    __syncthreads();
-    const uint32_t natoms = min(8u, atoms_per_rb - seg * 8);
-    uint8_t *dst = p.sf + ((int64_t)((p.sf_row0 >> 7) + rb) * atoms_per_rb + seg * 8) * 512;
-    for (uint32_t t = threadIdx.x; t < natoms * 32; t += blockDim.x)
-      reinterpret_cast<uint4 *>(dst)[t] = reinterpret_cast<const uint4 *>(sf_tile)[t];
-    __syncthreads();
+    return;
+  }
+  // ---------------------------------------------------------------- encoders
+  const int cw = warp - 1;
+  const int cb = lane % C::BPR, rsub = lane / C::BPR;
+  const EncodeConsts kc = encode_consts(p.gscale);
+  // per-lane offsets that do not change from unit to unit: this lane's rows
+  // of the unit (codes: row * K/2) and their places in the scale atoms
+  int64_t code_off[C::SPW];
+  int sf_off[C::SPW];
+#pragma unroll
+  for (int j = 0; j < C::SPW; ++j) {
+    const int r = (cw * C::SPW + j) * C::RPS + rsub;
+    code_off[j] = (int64_t)r * (p.K >> 1);
+    sf_off[j] = (r & 31) * 16 + (r >> 5) * 4 + (cb & 3);
+  }
+  const int64_t atoms_per_rb = p.K >> 6;
+  int st = 0;
+  uint32_t ph = 0;
+  for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const uint32_t rb = u / nseg, seg = u - rb * nseg;
+    if (!mbar_wait(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
+    const T *sx = reinterpret_cast<const T *>(ring + st * C::STAGE_BYTES) + rsub * C::COLS + cb * 16;
+    const int64_t gcol = (int64_t)seg * C::COLS + cb * 16;
+    const bool col_ok = gcol < p.K;
+    const int64_t row0 = (int64_t)rb * 128;
+    uint8_t *codes_u = p.codes + row0 * (p.K >> 1) + (gcol >> 1);
+    uint8_t *sf_u = p.sf + (((p.sf_row0 >> 7) + rb) * atoms_per_rb + (gcol >> 6)) * 512;
+    Block16<T> in[C::SPW];
+#pragma unroll
+    for (int j = 0; j < C::SPW; ++j) in[j].load_shared(sx + (cw * C::SPW + j) * C::RPS * C::COLS);
+#pragma unroll
+    for (int j = 0; j < C::SPW; ++j) {
+      const int r = (cw * C::SPW + j) * C::RPS + rsub;
+      uint32_t s;
+      const uint2 word = encode16(in[j], kc, rcp_tab, sx + (cw * C::SPW + j) * C::RPS * C::COLS, &s);
+      if (col_ok) {
+        if (row0 + r < p.rows) *reinterpret_cast<uint2 *>(codes_u + code_off[j]) = word;
+        sf_u[sf_off[j]] = (uint8_t)s;
+      }
+    }
+    // this warp is done with the stage (its reads happen-before the arrive)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+    if (++st == C::STAGES) { st = 0; ph ^= 1; }
   }
 }
 
@@ -349,18 +458,16 @@ __global__ void __launch_bounds__(256) quantize_tile_kernel(QuantizeParams p) {
 template <typename T>
 __global__ void __launch_bounds__(256) amax_kernel(const T *x, int64_t rows, int64_t K, int64_t ld,
                                                    unsigned *amax_bits) {
-  const int64_t chunks_per_row = K >> 3;
+  pdl_prologue();
+  const int64_t chunks_per_row = K >> 4;
   const int64_t n = rows * chunks_per_row;
   float m = 0.0f;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / chunks_per_row, c = (i - r * chunks_per_row) * 8;
-    Vec8<T> v8;
-    v8.load(x + r * ld + c);
-    float v[8];
-    v8.to_f32(v);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    const int64_t r = i / chunks_per_row, c = (i - r * chunks_per_row) * 16;
+    Block16<T> b;
+    b.load(x + r * ld + c);
+    m = fmaxf(m, b.amax());
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));

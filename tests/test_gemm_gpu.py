@@ -107,6 +107,9 @@ def _random_case(M, N, K, seed, out_dtype, a_dtype=torch.bfloat16):
     (200, 300, 320),      # ragged M and N, K not a multiple of 256
     (129, 96, 5120),      # small N (128-wide tile), split-K
     (384, 1000, 1344),    # ragged everything, several waves of stages
+    (100, 2000, 1344),    # activation as the 128-wide MMA N, K tail, cluster split-K
+    (1000, 40, 832),      # weight as a 64-wide MMA N, cluster split-K
+    (700, 20, 768),       # weight as a 32-wide MMA N
 ])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_gemm_shapes(M, N, K, out_dtype):

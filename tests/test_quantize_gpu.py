@@ -44,7 +44,7 @@ def test_tiny_fp32():
     _quant_check(W.make_w(wl, 0))
 
 
-@pytest.mark.parametrize("rows,K", [(1, 64), (33, 192), (127, 320), (129, 256), (300, 576)])
+@pytest.mark.parametrize("rows,K", [(1, 64), (33, 192), (127, 320), (129, 256), (300, 576), (4096, 2048)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_ragged_shapes(rows, K, dtype):
     x = W.gaussian(rows, K, seed=rows * 7 + K, outliers=W.Outliers("scale", 0.05, 40.0), dtype=dtype)
