@@ -165,6 +165,15 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float
  *   y        : [M, N] (y_dt), row stride ld_y (device).
  *   workspace: device scratch, >= w4a4_gemm_workspace_bytes(M, N, K) bytes;
  *              holds the quantized activation and any split-K partial sums.
+ * Launch behaviour: the quantize and the GEMM are enqueued with programmatic
+ * stream serialization.  The quantize waits for the stream's preceding work
+ * before it reads x; the GEMM may start while the quantize runs and loads
+ * the weight (w_codes, w_sf) before it waits for the quantize.  Weights
+ * written by earlier work on the stream are therefore safe, since that work
+ * finishes before the quantize lets the GEMM start.  Do not rewrite the
+ * weight with a kernel that is still running when w4a4_gemm is enqueued (a
+ * kernel that itself let later grids start early); use an event between
+ * the two instead.
  */
 size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,

@@ -12,9 +12,13 @@
 //              on the preceding kernel (the weight) are issued first, then
 //              the thread waits for that kernel (programmatic dependent
 //              launch) before loading the activation side.
-//   warp 1     TMEM allocation and MMA issue: tcgen05.cp of the scale atoms,
-//              four tcgen05.mma kind::mxf4nvf4 (K = 64) per stage.
-//   warps 2-5  epilogue: each CTA owns a share of the output tile (whole
+//   warp 1     TMEM allocation and MMA issue: four tcgen05.mma
+//              kind::mxf4nvf4 (K = 64) per stage and nothing else.
+//   warps 2-5  during the K loop, scale warps (one per TMEM lane quarter):
+//              they move each stage's scale atoms from shared memory into
+//              the stage's TMEM columns with tcgen05.st (the replicated image
+//              a 32x128b.warpx4 copy would make), which keeps the MMA thread
+//              from issuing two copies per MMA.  Then the epilogue: each CTA owns a share of the output tile (whole
 //              output columns for decode, whole rows otherwise); the FP32
 //              partial tile leaves TMEM and every element is stored straight
 //              into the owner CTA's shared memory, in the slot of the
@@ -51,14 +55,12 @@ struct ClusterCfg {
   static constexpr int TMEM_COLS = TMEM_NEEDED <= 64 ? 64 : TMEM_NEEDED <= 128 ? 128
                                   : TMEM_NEEDED <= 256 ? 256 : 512;
   static constexpr int MAX_SPLITS = 8;
-  // reduction slots: S slots, each one owner share: ceil(BN/S) columns of
-  // 128 floats, or ceil(128/S) rows of BN+1 floats (S * ceil(D/S) <= D+S-1)
-  static constexpr int RED_PITCH = BN + 1;                  // odd: conflict-free rows and columns
-  static constexpr int RED_NEED = (BN + MAX_SPLITS - 1) * BM > (BM + MAX_SPLITS - 1) * RED_PITCH
-                                      ? (BN + MAX_SPLITS - 1) * BM
-                                      : (BM + MAX_SPLITS - 1) * RED_PITCH;
-  static constexpr int RED_FLOATS = (RED_NEED + 31) / 32 * 32;   // keeps the barriers after it 128-byte aligned
+  // reduction slots: S slots, each one owner's share of ceil(128/S) tile rows
+  // of RED_PITCH floats (16-byte rows for vector stores); S*ceil(128/S) <= 135
+  static constexpr int RED_PITCH = BN + 4;
+  static constexpr int RED_FLOATS = ((BM + MAX_SPLITS - 1) * RED_PITCH + 31) / 32 * 32;   // 128-byte multiple
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RED_FLOATS * 4 + 256;
+  static_assert((3 * STAGES + 2) * 8 + 8 <= 256, "barrier area");
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                     ((uint32_t)(BM >> 4) << 24);
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 128, "MMA N");
@@ -86,7 +88,8 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(red + C::RED_FLOATS);
   uint64_t *full = bars;
   uint64_t *empty = bars + C::STAGES;
-  uint64_t *tfull = bars + 2 * C::STAGES;
+  uint64_t *sfready = bars + 2 * C::STAGES;     // the stage's scales are in TMEM (4 warps)
+  uint64_t *tfull = bars + 3 * C::STAGES;
   uint64_t *tdone = tfull + 1;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tfull + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -106,6 +109,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfready[s], C::EPI_WARPS);
     }
     mbar_init(tfull, 1);
     mbar_init(tdone, 1);
@@ -191,33 +195,22 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       // ------------------------------------------------------------- MMA issue
       const uint64_t a_desc0 = smem_desc(smem_u32(sA), 16, 1024, 2);
       const uint64_t b_desc0 = smem_desc(smem_u32(sB), 16, 1024, 2);
-      const uint64_t sfa_desc0 = smem_desc(smem_u32(sSFA), 0, 128, 0);
-      const uint64_t sfb_desc0 = smem_desc(smem_u32(sSFB), 0, 128, 0);
       int st = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int ks = ks0; ks < ks1; ++ks) {
-        if (!mbar_wait(&full[st], ph, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&sfready[st], ph, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint64_t ad = a_desc0 + (uint64_t)((st * C::A_BYTES) >> 4);
         const uint64_t bd = b_desc0 + (uint64_t)((st * C::B_BYTES) >> 4);
-        const uint64_t sad = sfa_desc0 + (uint64_t)((st * C::SFA_BYTES) >> 4);
-        const uint64_t sbd = sfb_desc0 + (uint64_t)((st * C::SFB_BYTES) >> 4);
         const uint32_t reg = tmem + (uint32_t)(st * C::SF_COLS);
         const int nkb = min(4, p.kblocks - ks * 4);
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          if (kb < nkb) {
-            tc_cp_32x128b_warpx4(reg + C::SFA_COL + 4 * kb, sad + (uint64_t)(kb * 32));
-#pragma unroll
-            for (int j = 0; j < C::SFB_ATOMS; ++j)
-              tc_cp_32x128b_warpx4(reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS + 4 * j,
-                                   sbd + (uint64_t)(j * 128 + kb * 32));
+        for (int kb = 0; kb < 4; ++kb)
+          if (kb < nkb)
             tc_mma_nvfp4(tmem, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), C::IDESC,
                          (ks > ks0 || kb > 0) ? 1u : 0u, reg + C::SFA_COL + 4 * kb,
                          reg + C::SFB_COL + kb * 4 * C::SFB_ATOMS);
-          }
-        }
         tc_commit(&empty[st]);
         if (++st == C::STAGES) { st = 0; ph ^= 1; }
       }
@@ -228,18 +221,59 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       mbar_wait(tdone, 0, p.err, ERR_MMA, &never);
     }
   } else {
-    // ------------------------------- epilogue: partial tile -> owners' slots
     const int q = warp & 3;                       // TMEM lane quarter of this warp
     const int i = q * 32 + lane;                  // tile row (A row)
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    {
+      // ----------------------------------------------------- scale warps
+      // Lane l writes, for each 64-deep K block kb of the stage, the 16-byte
+      // line l of the A atom and of the B atom(s) into its TMEM lane 32q + l:
+      // columns SFA_COL + 4kb .. +3 and SFB_COL + 4kb*SFB_ATOMS .. (the
+      // layout the MMA reads).  A stage's columns are rewritten only after
+      // its next load has landed, i.e. after the MMAs that read them.
+      int st = 0;
+      uint32_t ph = 0;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        if (!mbar_wait(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
+        const uint4 *sa = reinterpret_cast<const uint4 *>(sSFA + st * C::SFA_BYTES) + lane;
+        const uint4 *sb = reinterpret_cast<const uint4 *>(sSFB + st * C::SFB_BYTES) + lane;
+        const uint32_t reg = tmem + lane_addr + (uint32_t)(st * C::SF_COLS);
+        uint32_t ra[16];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          const uint4 a = sa[kb * 32];
+          ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
+        }
+        tmem_st16(reg + C::SFA_COL, ra);
+#pragma unroll
+        for (int h = 0; h < C::SFB_ATOMS; ++h) {
+          // B region, 4*SFB_ATOMS words per K block: atom j of the K block at 4j
+          uint32_t rb[16];
+#pragma unroll
+          for (int w = 0; w < 16; ++w) {
+            const int kb = (h * 16 + w) / (4 * C::SFB_ATOMS), j = ((h * 16 + w) / 4) % C::SFB_ATOMS;
+            const uint4 b = sb[j * 128 + kb * 32];
+            rb[w] = (w & 3) == 0 ? b.x : ((w & 3) == 1 ? b.y : ((w & 3) == 2 ? b.z : b.w));
+          }
+          tmem_st16(reg + C::SFB_COL + 16 * h, rb);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfready[st]);
+        if (++st == C::STAGES) { st = 0; ph ^= 1; }
+      }
+    }
+    // ------------------------------- epilogue: partial tile -> owners' slots
+    // Tile row i belongs to rank i*S/128, whose share starts at ceil(r*128/S);
+    // slots are one share (ceil(128/S) rows) apart.
     const bool ok = mbar_wait(tfull, 0, p.err, ERR_EPILOGUE, abort_flag);
     if (ok) tc_fence_after();
-    const uint32_t red_base = smem_u32(red);
-    // shares: index x of a dimension of size D belongs to rank x*S/D, whose
-    // share starts at ceil(r*D/S); slots are one share apart
-    const uint32_t slot = i_fast ? (uint32_t)((BN + S - 1) / S * C::BM) : (uint32_t)((C::BM + S - 1) / S * C::RED_PITCH);
+    const uint32_t slot = (uint32_t)((C::BM + S - 1) / S * C::RED_PITCH);
     const int own_r = i * S / C::BM;
     const int row0_r = (own_r * C::BM + S - 1) / S;
+    const uint32_t dst = mapa_shared(smem_u32(red) + (rank * slot + (uint32_t)((i - row0_r) * C::RED_PITCH)) * 4u,
+                                     (uint32_t)own_r);
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t acc[32];
@@ -250,45 +284,31 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) acc[e] = 0u;
       }
-      if (i_fast) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = c + e;
-          const int r = j * S / BN;
-          const int j0 = (r * BN + S - 1) / S;
-          const uint32_t off = (rank * slot + (uint32_t)((j - j0) * C::BM + i)) * 4u;
-          st_shared_cluster_f32(mapa_shared(red_base + off, (uint32_t)r), __uint_as_float(acc[e]));
-        }
-      } else {
-        const uint32_t dst =
-            mapa_shared(red_base + (rank * slot + (uint32_t)((i - row0_r) * C::RED_PITCH + c)) * 4u, (uint32_t)own_r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) st_shared_cluster_f32(dst + 4u * e, __uint_as_float(acc[e]));
-      }
+      for (int e = 0; e < 32; e += 4) st_shared_cluster_v4(dst + 4u * (c + e), acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
     }
   }
 
   // ------------------------------------------------- cluster-wide reduction
   // After the barrier every slot of this CTA's share holds the partial of
-  // the rank it is named after; sum them in rank order.
+  // the rank it is named after; sum them in rank order.  Elements are dealt
+  // out in output order: tile row fastest when the tile row is the output's
+  // unit-stride index (decode), tile column fastest otherwise.
   __syncwarp();                   // reconverge the role warps (the cluster barrier is warp-aligned)
   tc_fence_before();
   cluster_sync();
   {
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
-    const int D = i_fast ? BN : C::BM;                      // the dimension shared out
-    const int inner = i_fast ? C::BM : BN;
-    const int first = (rank * D + S - 1) / S;
-    const int n_own = ((rank + 1) * D + S - 1) / S - first;
-    const int slot = i_fast ? (BN + S - 1) / S * C::BM : (C::BM + S - 1) / S * C::RED_PITCH;
-    const int E = n_own * inner;
+    const int first = (rank * C::BM + S - 1) / S;
+    const int n_rows = ((rank + 1) * C::BM + S - 1) / S - first;
+    const int slot = (C::BM + S - 1) / S * C::RED_PITCH;
+    const int E = n_rows * BN;
     for (int e = (int)threadIdx.x; e < E; e += C::THREADS) {
-      const int a = e / inner, b = e - a * inner;          // (owned column, row) or (owned row, column)
-      const int i = i_fast ? b : first + a;
-      const int j = i_fast ? first + a : b;
-      const int gi = ta * C::BM + i, gj = tb * BN + j;
+      const int a = i_fast ? e % n_rows : e / BN;          // row within the share
+      const int j = i_fast ? e / n_rows : e % BN;
+      const int gi = ta * C::BM + first + a, gj = tb * BN + j;
       if (gi >= p.rows_a || gj >= p.rows_b) continue;
-      const int off = i_fast ? a * C::BM + b : a * C::RED_PITCH + b;
+      const int off = a * C::RED_PITCH + j;
       float acc = red[off];
 #pragma unroll
       for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
