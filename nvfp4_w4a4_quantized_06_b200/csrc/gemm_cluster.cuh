@@ -291,9 +291,8 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
 
   // ------------------------------------------------- cluster-wide reduction
   // After the barrier every slot of this CTA's share holds the partial of
-  // the rank it is named after; sum them in rank order.  Elements are dealt
-  // out in output order: tile row fastest when the tile row is the output's
-  // unit-stride index (decode), tile column fastest otherwise.
+  // the rank it is named after; sum them in rank order.  Lanes run along the
+  // output's unit-stride index: the tile row for decode, the column otherwise.
   __syncwarp();                   // reconverge the role warps (the cluster barrier is warp-aligned)
   tc_fence_before();
   cluster_sync();
@@ -302,21 +301,25 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
     const int first = (rank * C::BM + S - 1) / S;
     const int n_rows = ((rank + 1) * C::BM + S - 1) / S - first;
     const int slot = (C::BM + S - 1) / S * C::RED_PITCH;
-    const int E = n_rows * BN;
-    for (int e = (int)threadIdx.x; e < E; e += C::THREADS) {
-      const int a = i_fast ? e % n_rows : e / BN;          // row within the share
-      const int j = i_fast ? e / n_rows : e % BN;
-      const int gi = ta * C::BM + first + a, gj = tb * BN + j;
-      if (gi >= p.rows_a || gj >= p.rows_b) continue;
-      const int off = a * C::RED_PITCH + j;
-      float acc = red[off];
+    // warps step over one index, lanes over the output's unit-stride one
+    const int nw = C::THREADS / 32;
+    const int outer_n = i_fast ? BN : n_rows, inner_n = i_fast ? n_rows : BN;
+    for (int o1 = warp; o1 < outer_n; o1 += nw) {
+      for (int o2 = lane; o2 < inner_n; o2 += 32) {
+        const int a = i_fast ? o2 : o1;                      // row within the share
+        const int j = i_fast ? o1 : o2;
+        const int gi = ta * C::BM + first + a, gj = tb * BN + j;
+        if (gi >= p.rows_a || gj >= p.rows_b) continue;
+        const int off = a * C::RED_PITCH + j;
+        float acc = red[off];
 #pragma unroll
-      for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
-        if (s2 < S) acc = acc + red[s2 * slot + off];
-      const float v = __fmul_rn(acc, alpha);
-      const int64_t o = (int64_t)gi * p.out_si + (int64_t)gj * p.out_sj;
-      if constexpr (MODE == OUT_BF16) static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(v);
-      else static_cast<float *>(p.out)[o] = v;
+        for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
+          if (s2 < S) acc = acc + red[s2 * slot + off];
+        const float v = __fmul_rn(acc, alpha);
+        const int64_t o = (int64_t)gi * p.out_si + (int64_t)gj * p.out_sj;
+        if constexpr (MODE == OUT_BF16) static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(v);
+        else static_cast<float *>(p.out)[o] = v;
+      }
     }
   }
   __syncwarp();

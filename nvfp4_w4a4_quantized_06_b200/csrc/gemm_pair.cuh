@@ -14,15 +14,15 @@
 // Scale factors reach TMEM through tcgen05.st, not tcgen05.cp: the NVFP4
 // scales of a 128 x 256 x 256 slice are 24 KB of replicated TMEM columns per
 // SM per stage, which the smem->TMEM copy path moves at ~40 B/clk (slower
-// than the MMAs that consume them), while four "scale warps" (one per TMEM
-// lane quarter) store them from registers at several hundred B/clk and leave
-// the single MMA-issuing thread nothing but MMAs.
+// than the MMAs that consume them), while eight "scale warps" (per TMEM lane
+// quarter one for the A scales and one for the B scales) store them from
+// registers at several hundred B/clk and leave the single MMA-issuing thread
+// nothing but MMAs.
 //
 // Warp roles per CTA: 0 producer (one lane), 1 TMEM allocation + MMA issue
-// (one lane of the leader), 2-5 scale warps (lane quarters 2, 3, 0, 1), 6-21
-// epilogue (four warps per lane quarter, 64 columns each).  22 warps fit one
-// SM at <= 80 registers per thread (registers are split across the four
-// schedulers: 6 warps x 32 x 80 <= 16K each).
+// (one lane of the leader), 2-5 A-scale warps and 6-9 B-scale warps (lane
+// quarters 2, 3, 0, 1), 10-25 epilogue (four warps per lane quarter, 64
+// columns each).  26 warps fit one SM at <= 72 registers per thread.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -42,7 +42,7 @@ struct PairCfg {
   static constexpr int SFB_BYTES = 2 * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = 5;
-  static constexpr int SF_WARPS = 4;
+  static constexpr int SF_WARPS = 8;
   static constexpr int EPI_WARPS = 16;
   static constexpr int EPI_COLS = 64;            // four warps per lane quarter, 64 columns each
   static constexpr int FIRST_EPI_WARP = 2 + SF_WARPS;
@@ -203,11 +203,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     }
   } else if (warp < C::FIRST_EPI_WARP) {
     // ----------------------------------------------------------- scale warps
-    // Lane l of the warp for lane quarter q writes, for every 64-deep K block,
-    // the 16 bytes of line l of the A atom (scales of rows l, l+32, l+64,
-    // l+96 of this CTA) and of the two B atoms into its TMEM lane 32q + l --
-    // the same replicated image a 32x128b.warpx4 copy would produce.
+    // Warps 2-5 write the A scales, warps 6-9 the B scales, each for the TMEM
+    // lane quarter warp % 4: lane l writes line l of the atoms into lane 32q + l.
     const int q = warp & 3;
+    const bool a_role = warp < 6;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const uint32_t ready_leader = mapa_shared(smem_u32(&sfready[0]), 0);
     int st = 0;
@@ -216,25 +215,31 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       for (int ks = 0; ks < p.kstages; ++ks) {
         uint64_t *bar = leader ? &full[st] : &sffull[st];
         if (!mbar_wait(bar, ph, p.err, ERR_MMA, abort_flag)) { u = total_units; break; }
-        const uint4 *sa = reinterpret_cast<const uint4 *>(sSFA + st * C::SFA_BYTES) + lane;
-        const uint4 *sb = reinterpret_cast<const uint4 *>(sSFB + st * C::SFB_BYTES) + lane;
-        uint32_t ra[16], rb0[16], rb1[16];
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          const uint4 a = sa[kb * 32];             // atom kb, line `lane`
-          const uint4 b0 = sb[kb * 32];            // B rows 0..127, atom kb
-          const uint4 b1 = sb[128 + kb * 32];      // B rows 128..255, atom kb
-          ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
-          // B region, 8 words per K block: atom of rows 0..127, then rows 128..255
-          uint32_t *bw = kb < 2 ? rb0 : rb1;
-          const int o = (kb & 1) * 8;
-          bw[o] = b0.x; bw[o + 1] = b0.y; bw[o + 2] = b0.z; bw[o + 3] = b0.w;
-          bw[o + 4] = b1.x; bw[o + 5] = b1.y; bw[o + 6] = b1.z; bw[o + 7] = b1.w;
-        }
         const uint32_t reg = tmem + lane_addr + (uint32_t)(st * C::SF_COLS);
-        tmem_st16(reg + C::SFA_COL, ra);
-        tmem_st16(reg + C::SFB_COL, rb0);
-        tmem_st16(reg + C::SFB_COL + 16, rb1);
+        if (a_role) {
+          const uint4 *sa = reinterpret_cast<const uint4 *>(sSFA + st * C::SFA_BYTES) + lane;
+          uint32_t ra[16];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 a = sa[kb * 32];
+            ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
+          }
+          tmem_st16(reg + C::SFA_COL, ra);
+        } else {
+          const uint4 *sb = reinterpret_cast<const uint4 *>(sSFB + st * C::SFB_BYTES) + lane;
+          uint32_t rb0[16], rb1[16];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 b0 = sb[kb * 32];
+            const uint4 b1 = sb[128 + kb * 32];
+            uint32_t *bw = kb < 2 ? rb0 : rb1;
+            const int o = (kb & 1) * 8;
+            bw[o] = b0.x; bw[o + 1] = b0.y; bw[o + 2] = b0.z; bw[o + 3] = b0.w;
+            bw[o + 4] = b1.x; bw[o + 5] = b1.y; bw[o + 6] = b1.z; bw[o + 7] = b1.w;
+          }
+          tmem_st16(reg + C::SFB_COL, rb0);
+          tmem_st16(reg + C::SFB_COL + 16, rb1);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
