@@ -301,8 +301,11 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
   const uint32_t nseg = (uint32_t)((p.K + 511) >> 9);
   const uint32_t units = (uint32_t)p.rows * nseg;
   const int64_t ncols = p.K >> 4;
-  const EncodeConsts kc = encode_consts(p.gscale);
   const T *x = static_cast<const T *>(p.x);
+  // the encoder constants are read after the first loads are in flight, so
+  // the two round trips overlap (few-row calls run a single iteration)
+  EncodeConsts kc;
+  bool have_kc = false;
 
   for (uint32_t u0 = warp * UNROLL; u0 < units; u0 += nwarps * UNROLL) {
     Block16<T> in[UNROLL];
@@ -315,6 +318,10 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
       col[j] = (int)(u - (uint32_t)row[j] * nseg) * 512 + lane * 16;
       in[j].zero();
       if (u < units && col[j] < p.K) in[j].load(x + row[j] * p.ld_x + col[j]);
+    }
+    if (!have_kc) {
+      kc = encode_consts(p.gscale);
+      have_kc = true;
     }
 #pragma unroll
     for (int j = 0; j < UNROLL; ++j) {
