@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++it) {
       int ta, tb, split;
       unit_coords(p, u, ta, tb, split);
-      if (!mbar_wait(tfull, it & 1, p.err, ERR_EPILOGUE, abort_flag)) break;
+      if (!mbar_wait_warp(tfull, it & 1, p.err, ERR_EPILOGUE, abort_flag)) break;
       tc_fence_after();
       uint32_t acc[C::EPI_COLS];
 #pragma unroll

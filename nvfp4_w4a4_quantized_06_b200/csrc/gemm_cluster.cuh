@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       int st = 0;
       uint32_t ph = 0;
       for (int ks = ks0; ks < ks1; ++ks) {
-        if (!mbar_wait(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
+        if (!mbar_wait_warp(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
         const uint4 *sa = reinterpret_cast<const uint4 *>(sSFA + st * C::SFA_BYTES) + lane;
         const uint4 *sb = reinterpret_cast<const uint4 *>(sSFB + st * C::SFB_BYTES) + lane;
         const uint32_t reg = tmem + lane_addr + (uint32_t)(st * C::SF_COLS);
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
     // ------------------------------- epilogue: partial tile -> owners' slots
     // Tile row i belongs to rank i*S/128, whose share starts at ceil(r*128/S);
     // slots are one share (ceil(128/S) rows) apart.
-    const bool ok = mbar_wait(tfull, 0, p.err, ERR_EPILOGUE, abort_flag);
+    const bool ok = mbar_wait_warp(tfull, 0, p.err, ERR_EPILOGUE, abort_flag);
     if (ok) tc_fence_after();
     const uint32_t slot = (uint32_t)((C::BM + S - 1) / S * C::RED_PITCH);
     const int own_r = i * S / C::BM;

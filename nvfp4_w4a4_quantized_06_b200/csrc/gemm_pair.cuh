@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     for (int u = cluster; u < total_units; u += nclusters) {
       for (int ks = 0; ks < p.kstages; ++ks) {
         uint64_t *bar = leader ? &full[st] : &sffull[st];
-        if (!mbar_wait(bar, ph, p.err, ERR_MMA, abort_flag)) { u = total_units; break; }
+        if (!mbar_wait_warp(bar, ph, p.err, ERR_MMA, abort_flag)) { u = total_units; break; }
         const uint32_t reg = tmem + lane_addr + (uint32_t)(st * C::SF_COLS);
         if (a_role) {
           const uint4 *sa = reinterpret_cast<const uint4 *>(sSFA + st * C::SFA_BYTES) + lane;
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     for (int u = cluster; u < total_units; u += nclusters, ++it) {
       int ta, tb, split;
       unit_coords(p, u, ta, tb, split);
-      if (!mbar_wait(tfull, it & 1, p.err, ERR_EPILOGUE, abort_flag)) break;
+      if (!mbar_wait_warp(tfull, it & 1, p.err, ERR_EPILOGUE, abort_flag)) break;
       tc_fence_after();
       const int i = ta * 256 + (int)rank * C::BM + q * 32 + lane;
       const int j0 = tb * C::BN + cbase;

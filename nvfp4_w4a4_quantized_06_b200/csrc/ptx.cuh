@@ -88,6 +88,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
   }
 }
 
+// The same wait executed by all 32 lanes of a warp, with one verdict for the
+// whole warp, so that a timeout never leaves some lanes of a warp ahead of
+// the others (the warp-wide tcgen05 and barrier instructions that follow
+// need the full warp).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, unsigned *err, unsigned code,
+                                               volatile int *abort_flag) {
+  const bool ok = mbar_wait(bar, parity, err, code, abort_flag);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
 // ----------------------------------------------------------------------- TMA
 // 2D tiled load of a box into shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, uint64_t *bar,

@@ -345,30 +345,30 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
 
 // Streaming path for calls whose scale rows start on a 128-row boundary and
 // that own every row of their last 128-row block (the activation quantize
-// always does).  One CTA per SM, persistent over units of 128 rows x COLS
-// columns (64 KB of input; COLS = 256 bf16 / 128 fp32):
-//   warp 0       one thread streams units into a ring of shared-memory stages
-//                with 2D TMA loads (rows past `rows` and columns past K read
-//                as zeros, so padding rows get zero scales);
-//   warps 1..16  encode: lane l takes block l % (COLS/16) of row
-//                l / (COLS/16) of each step and writes its 8 code bytes and
-//                its scale byte straight to global memory (a warp's scale
-//                bytes fill 4-byte runs of the swizzled atoms, which the L2
-//                merges); each warp hands the stage back on its own, so the
-//                warps never wait for one another.
+// always does).  One CTA of 32 warps per SM, persistent over units of 128
+// rows x COLS columns (64 KB of input; COLS = 256 bf16 / 128 fp32) that
+// stream through a ring of shared-memory stages by 2D TMA (rows past `rows`
+// and columns past K read as zeros, so padding rows get zero scales).  Every
+// warp encodes: lane l takes block l % (COLS/16) of row l / (COLS/16) of
+// each step and writes its 8 code bytes and its scale byte straight to
+// global memory (a warp's scale bytes fill 4-byte runs of the swizzled atoms,
+// which the L2 merges).  Each warp hands a stage back on its own; lane 0 of
+// warp 0 also refills it, once all 32 warps have, with the unit STAGES
+// ahead.  No warp is set aside for loading, so all 32 warps issue encoder
+// work (the encoder is issue-bound).
 template <typename T>
 struct QTmaCfg {
   static constexpr int ROWS = 128;
   static constexpr int COLS = sizeof(T) == 2 ? 256 : 128;
   static constexpr int BPR = COLS / 16;                 // blocks per row
   static constexpr int RPS = 32 / BPR;                  // rows per warp step
-  static constexpr int CONSUMERS = 16;
-  static constexpr int SPW = ROWS / RPS / CONSUMERS;    // steps per warp per unit
+  static constexpr int WARPS = 32;
+  static constexpr int SPW = ROWS / RPS / WARPS;        // steps per warp per unit
   static constexpr int STAGE_BYTES = ROWS * COLS * (int)sizeof(T);
   static constexpr int STAGES = 3;
-  static constexpr int THREADS = 32 * (1 + CONSUMERS);
+  static constexpr int THREADS = 32 * WARPS;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * STAGES * 8 + 512 + 16;
-  static_assert(ROWS % (RPS * CONSUMERS) == 0, "unit split");
+  static_assert(ROWS % (RPS * WARPS) == 0 && SPW >= 1, "unit split");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -387,10 +387,16 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t nseg = (uint32_t)((p.K + C::COLS - 1) / C::COLS);
   const uint32_t units = (uint32_t)((p.rows + 127) >> 7) * nseg;
-  if (threadIdx.x == 0) {
+  const bool loader = threadIdx.x == 0;
+  auto issue = [&](int st, uint32_t u) {
+    const uint32_t rb = u / nseg, seg = u - rb * nseg;
+    mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+    tma_load_2d(ring + st * C::STAGE_BYTES, &tmx, &full[st], (int32_t)(seg * C::COLS), (int32_t)(rb * 128));
+  };
+  if (loader) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::CONSUMERS);
+      mbar_init(&empty[s], C::WARPS);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -399,24 +405,14 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   fill_rcp_table(rcp_tab);
   pdl_prologue();
   __syncthreads();
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      int st = 0;
-      uint32_t ph = 0;
-      for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
-        if (!mbar_wait(&empty[st], ph ^ 1, p.err, ERR_PRODUCER, abort_flag)) break;
-        const uint32_t rb = u / nseg, seg = u - rb * nseg;
-        mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-        tma_load_2d(ring + st * C::STAGE_BYTES, &tmx, &full[st], (int32_t)(seg * C::COLS), (int32_t)(rb * 128));
-        if (++st == C::STAGES) { st = 0; ph ^= 1; }
-      }
+  if (loader) {
+    // the first round of the ring (x is readable: the prologue has waited)
+    for (int s = 0; s < C::STAGES; ++s) {
+      const uint32_t u = blockIdx.x + (uint32_t)s * gridDim.x;
+      if (u < units) issue(s, u);
     }
-    return;
   }
-  // ---------------------------------------------------------------- encoders
-  const int cw = warp - 1;
+
   const int cb = lane % C::BPR, rsub = lane / C::BPR;
   const EncodeConsts kc = encode_consts(p.gscale);
   // per-lane offsets that do not change from unit to unit: this lane's rows
@@ -425,7 +421,7 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   int sf_off[C::SPW];
 #pragma unroll
   for (int j = 0; j < C::SPW; ++j) {
-    const int r = (cw * C::SPW + j) * C::RPS + rsub;
+    const int r = (warp * C::SPW + j) * C::RPS + rsub;
     code_off[j] = (int64_t)r * (p.K >> 1);
     sf_off[j] = (r & 31) * 16 + (r >> 5) * 4 + (cb & 3);
   }
@@ -434,7 +430,7 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   uint32_t ph = 0;
   for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
     const uint32_t rb = u / nseg, seg = u - rb * nseg;
-    if (!mbar_wait(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
+    if (!mbar_wait_warp(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
     const T *sx = reinterpret_cast<const T *>(ring + st * C::STAGE_BYTES) + rsub * C::COLS + cb * 16;
     const int64_t gcol = (int64_t)seg * C::COLS + cb * 16;
     const bool col_ok = gcol < p.K;
@@ -443,12 +439,12 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
     uint8_t *sf_u = p.sf + (((p.sf_row0 >> 7) + rb) * atoms_per_rb + (gcol >> 6)) * 512;
     Block16<T> in[C::SPW];
 #pragma unroll
-    for (int j = 0; j < C::SPW; ++j) in[j].load_shared(sx + (cw * C::SPW + j) * C::RPS * C::COLS);
+    for (int j = 0; j < C::SPW; ++j) in[j].load_shared(sx + (warp * C::SPW + j) * C::RPS * C::COLS);
 #pragma unroll
     for (int j = 0; j < C::SPW; ++j) {
-      const int r = (cw * C::SPW + j) * C::RPS + rsub;
+      const int r = (warp * C::SPW + j) * C::RPS + rsub;
       uint32_t s;
-      const uint2 word = encode16(in[j], kc, rcp_tab, sx + (cw * C::SPW + j) * C::RPS * C::COLS, &s);
+      const uint2 word = encode16(in[j], kc, rcp_tab, sx + (warp * C::SPW + j) * C::RPS * C::COLS, &s);
       if (col_ok) {
         if (row0 + r < p.rows) *reinterpret_cast<uint2 *>(codes_u + code_off[j]) = word;
         sf_u[sf_off[j]] = (uint8_t)s;
@@ -457,6 +453,17 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
     // this warp is done with the stage (its reads happen-before the arrive)
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
+    bool stop = false;
+    if (loader) {
+      // refill the stage with this CTA's unit STAGES ahead once every warp
+      // has released it
+      const uint32_t un = u + (uint32_t)C::STAGES * gridDim.x;
+      if (un < units) {
+        if (mbar_wait(&empty[st], ph, p.err, ERR_PRODUCER, abort_flag)) issue(st, un);
+        else stop = true;
+      }
+    }
+    if (__any_sync(0xFFFFFFFFu, stop)) break;       // the whole warp leaves together
     if (++st == C::STAGES) { st = 0; ph ^= 1; }
   }
 }
