@@ -14,6 +14,9 @@ repair on the arxiv-wiki page ("접근 방법", "개발자 관점") and the abst
 shd-paper page.  Readings the pages leave open are listed in the C file's
 header.  Everything except the arithmetic order for non-power-of-two global
 scales is pinned by tests/test_oracle_*.py; that order is "parity unpinned".
+The rows marked "next" (GDN gate activations, fake-quant, FP8 KV quantize)
+follow the same pages (ta-paperlens "前提2"; arxiv-wiki "주요 결과") and are
+pinned in tests/test_oracle_next.py.
 """
 from __future__ import annotations
 
@@ -60,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_gemm_f64.argtypes, L.oracle_gemm_f64.restype = [vp, vp, i64, i64, i64, f64, vp, vp], None
         L.oracle_sf_gather.argtypes, L.oracle_sf_gather.restype = [vp, vp, i64, i64, vp], None
         L.oracle_num_threads.argtypes, L.oracle_num_threads.restype = [], i32
+        L.oracle_gdn_gates.argtypes, L.oracle_gdn_gates.restype = [vp, i64, i64, i64, vp], None
+        L.oracle_fp8_quantize.argtypes, L.oracle_fp8_quantize.restype = [vp, i64, f32, vp], None
         _lib = L
     return _lib
 
@@ -173,6 +178,36 @@ def linear_reference(x: np.ndarray, gx, w_codes: np.ndarray, w_sf: np.ndarray, g
     b = dequantize(w_codes, w_sf, 1.0)
     y, yabs = gemm_f64(a, b, float(np.float64(gx) * np.float64(gw)), brute=brute)
     return y, yabs, xc, xs
+
+
+# --------------------------------------------------- rows marked "next"
+def gdn_gates(y: np.ndarray, n_a: int) -> np.ndarray:
+    """alpha = exp(-softplus(y)) on columns [0, n_a), beta = sigmoid(y) on the
+    rest (float64; the gate-projection epilogue of a GDN layer)."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    rows, N = y.shape
+    out = np.empty_like(y)
+    lib().oracle_gdn_gates(_ptr(y), rows, N, int(n_a), _ptr(out))
+    return out
+
+
+def fake_quant(x: np.ndarray, g):
+    """Quantize then dequantize (Q -> DQ): the NVFP4 value every element of x
+    is replaced by (float64, exact), and the error statistics
+    (sum of squared error, sum of squared input)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    codes, sf = quantize(x, g)
+    dq = dequantize(codes, sf, g)
+    x64 = x.astype(np.float64)
+    return dq, float(np.sum((x64 - dq) ** 2)), float(np.sum(x64 ** 2))
+
+
+def fp8_quantize(x: np.ndarray, s) -> np.ndarray:
+    """FP8 E4M3 codes (sign in bit 7) of fl32(x / s), static per-tensor scale s."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    q = np.empty(x.shape, dtype=np.uint8)
+    lib().oracle_fp8_quantize(_ptr(x), x.size, float(np.float32(s)), _ptr(q))
+    return q
 
 
 def num_threads() -> int:

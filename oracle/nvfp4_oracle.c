@@ -276,3 +276,42 @@ void oracle_sf_gather(const uint8_t *sf, const int64_t *rows, int64_t nrows, int
         for (c = 0; c < K / ORACLE_BLOCK; ++c)
             out[i * (K / ORACLE_BLOCK) + c] = sf[oracle_sf_offset(rows[i], c, K)];
 }
+
+/* ---------------------------------------------- GDN gate activations (next) */
+
+/* The two gate projections of a GDN layer feed log-space gates (ta-paperlens
+ * page, "前提2"): the raw projection a_t goes through softplus and then the
+ * exponential to give alpha_t, how much of the state is kept (close to 1 =
+ * forget little), and b_t through the logistic sigmoid to give beta_t, the
+ * write strength.  The per-head decay scale and bias the model multiplies
+ * in are not on the pages, so this reading uses 1 and 0:
+ *   alpha = exp(-softplus(a)),  beta = 1 / (1 + exp(-b)),
+ * columns [0, n_a) of the fused gate GEMM output are a, the rest b.  float64. */
+static double softplus(double y)
+{
+    return y > 0.0 ? y + log1p(exp(-y)) : log1p(exp(y));
+}
+
+void oracle_gdn_gates(const double *y, int64_t rows, int64_t N, int64_t n_a, double *out)
+{
+    int64_t i;
+    for (i = 0; i < rows * N; ++i) {
+        double v = y[i];
+        out[i] = (i % N) < n_a ? exp(-softplus(v)) : 1.0 / (1.0 + exp(-v));
+    }
+}
+
+/* ------------------------------------------------ FP8 KV quantize (next) */
+
+/* Static per-tensor FP8 (E4M3) quantization of the KV cache (arxiv-wiki page,
+ * "주요 결과": a static per-tensor FP8 scale shipped with the checkpoint
+ * recovers most of the FP8 KV penalty): q = E4M3_RNE_SATFINITE(fl32(x / s))
+ * with the sign in bit 7; dequantization is dec(q) * s. */
+void oracle_fp8_quantize(const float *x, int64_t n, float s, uint8_t *q)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) {
+        float t = x[i] / s;      /* one IEEE fp32 division */
+        q[i] = (uint8_t)oracle_e4m3_encode(t);
+    }
+}
