@@ -116,8 +116,11 @@ def quantized_weight(wl, dev):
 
 
 def kernel_src_hash():
+    """Digest of the sources the CTA-pair GEMM is compiled from (its launch
+    shape lives in nvfp4w4a4.cu's plan; a change there that touches the pair
+    path must refresh profiles/dram_traffic.json by hand)."""
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh", "nvfp4w4a4.cu"):
+    for f in ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh"):
         h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_06_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -357,6 +360,57 @@ def measure_secondary(native, dev):
                      "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
                      "l2": f"CUDA graph over {copies} weight copies ({copies * wbytes / 1e6:.0f} MB)"}
         del g, wcs, wsfs, x, y, ws
+    # rows beyond the layer: fused gate epilogue, fake-quant, FP8 KV quantize
+    wl = W.WORKLOADS["gdn_gates_ab"]
+    x = W.make_x(wl).to(dev)
+    wc, wsf, gw = quantized_weight(wl, dev)
+    gx = native.amax_gscale(x)
+    out = torch.empty((wl.M, wl.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=12):
+        times = []
+        for i in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    ms = timed(lambda: native.gdn_gates(x, gx, wc, wsf, gw, n_a=wl.modules[0], out=out, workspace=ws))
+    byts = wl.M * wl.K * 2 + wl.N * wl.K // 2 + wl.N * wl.K // 16 + wl.M * wl.N * 4
+    res["gdn_gates_fused_activations"] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4),
+                                          "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                                          "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
+                                          "l2": "512 MB flush between reps"}
+    del x, wc, wsf, out, ws
+    wl = W.WORKLOADS["prefill_mlp_gate_up"]
+    x = W.make_x(wl).to(dev)
+    g = native.amax_gscale(x)
+    fq = torch.empty_like(x)
+    st = torch.empty(2, dtype=torch.float64, device=dev)
+    ms = timed(lambda: native.lib().nvfp4_fake_quant(x.data_ptr(), 0, wl.M, wl.K, wl.K, g.data_ptr(), fq.data_ptr(), 0,
+                                                     wl.K, st.data_ptr(), torch.cuda.current_stream().cuda_stream))
+    byts = wl.M * wl.K * 4
+    res["fake_quant_bf16"] = {"shape": f"{wl.M}x{wl.K}", "ms": round(ms, 4),
+                              "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
+                              "rel_error": round(float(np.sqrt(st[0].item() / st[1].item())), 5)}
+    del x, fq
+    kv = torch.randn(32 * 4096 * 4 * 256 * 2, dtype=torch.bfloat16, device=dev)     # 32 seqs x 4096 tokens, K and V
+    sc = (kv.abs().max().float() / 448.0).reshape(1)
+    q8 = torch.empty(kv.numel(), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: native.fp8_quantize(kv, sc, out=q8))
+    byts = kv.numel() * 3
+    res["fp8_kv_quantize"] = {"shape": "32x4096 tokens x 4 kv heads x 256 x (K,V) bf16", "ms": round(ms, 4),
+                              "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3)}
+    del kv, q8, flush
     assert native.last_device_status() == 0
     return res
 

@@ -217,6 +217,62 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
                                int64_t K, nvfp4_stream_t stream);
 
 /*
+ * ------------------------------------------------------------------------
+ * Rows beyond the layer itself, built on the same encoder and GEMM.
+ * ------------------------------------------------------------------------
+ *
+ * GDN gate projections with the gate activations fused into the GEMM
+ * epilogue (ta-paperlens page, "前提2": the raw projections a_t and b_t become
+ * alpha_t = exp(-softplus(a_t)), how much of the state is kept, and
+ * beta_t = sigmoid(b_t), the write strength; the model's per-head decay scale
+ * and bias are not part of this call: unit scale, zero bias).
+ *   x, x_gscale, w_codes, w_sf, w_gscale, workspace : as for w4a4_gemm; the
+ *              weight is the fused [a; b] gate projection (N <= 128 rows,
+ *              harmonized to one global scale when a and b were calibrated
+ *              apart).
+ *   gates    : [M, N] float32 (device), row stride ld_g: columns [0, n_a)
+ *              hold alpha, columns [n_a, N) hold beta.
+ * Errors: NVFP4_ERR_UNSUPPORTED when N > 128; otherwise as w4a4_gemm.  Same
+ * launch ordering as w4a4_gemm.
+ */
+nvfp4_status w4a4_gdn_gates(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                            const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, float *gates,
+                            int64_t ld_g, int64_t M, int64_t N, int64_t n_a, int64_t K, void *workspace,
+                            size_t workspace_bytes, nvfp4_stream_t stream);
+
+/*
+ * Fake-quant: every element of x replaced by the NVFP4 value it quantizes to,
+ * dec(q) * dec(s) * g (the values the W4A4 product sees; the pages measure
+ * the relative activation error this introduces, arxiv-wiki page, "주요 결과").
+ *   x        : [rows, K] bf16 or fp32, row stride ld_x (device).
+ *   gscale   : 1 float (device).
+ *   out      : [rows, K] bf16 or fp32 (out_dt), row stride ld_out (device);
+ *              FP32 output is the exact value rounded once to fp32, BF16 output
+ *              is that fp32 value rounded to bf16.
+ *   err_stats: NULL or 2 doubles (device, 8-byte aligned), overwritten with
+ *              [sum of (x - out)^2 in float64, sum of x^2]; the relative error
+ *              is sqrt(err_stats[0] / err_stats[1]).  The sums are accumulated
+ *              with atomics, so their rounding depends on timing (float64).
+ * Preconditions: K % 64 == 0; 16-byte aligned pointers and row strides.
+ */
+nvfp4_status nvfp4_fake_quant(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                              const float *gscale, void *out, nvfp4_out_dtype out_dt, int64_t ld_out,
+                              double *err_stats, nvfp4_stream_t stream);
+
+/*
+ * FP8 (E4M3) quantization with a static per-tensor scale, as used for the KV
+ * cache (arxiv-wiki page, "주요 결과": a static per-tensor FP8 KV scale shipped
+ * with the checkpoint recovers most of the FP8 KV penalty):
+ *   q[i] = E4M3_RNE_SATFINITE(fl32(x[i] / scale)), sign in bit 7
+ *   (dequantize as dec(q) * scale).
+ *   x     : n contiguous bf16 or fp32 values (device, 16-byte aligned), n % 8 == 0.
+ *   scale : 1 float (device), finite and > 0.
+ *   q     : n bytes (device, 8-byte aligned).
+ */
+nvfp4_status nvfp4_fp8_quantize(const void *x, nvfp4_in_dtype dt, int64_t n, const float *scale, uint8_t *q,
+                                nvfp4_stream_t stream);
+
+/*
  * Synchronizes the device, then reports and clears the library's device error
  * word: *flags receives the OR of the flags kernels recorded since the last
  * call (bit 0: a producer wait ran out, bit 1: an MMA wait ran out, bit 2: an

@@ -31,7 +31,9 @@
 
 namespace nvfp4 {
 
-enum OutMode : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_PARTIAL = 2 };
+// OUT_GATES: FP32 GDN gate activations of the fused a/b gate projection
+// (output columns [0, n_split) -> exp(-softplus(y)), the rest -> sigmoid(y)).
+enum OutMode : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_PARTIAL = 2, OUT_GATES = 3 };
 
 struct GemmParams {
   const uint8_t *sfa;
@@ -45,6 +47,7 @@ struct GemmParams {
   int kblocks;              // K / 64
   int kstages;              // ceil(K / 256)
   int tiles_a, tiles_b, splits, group;
+  int n_split;              // OUT_GATES: first output column of the b gates
   unsigned *err;
 };
 

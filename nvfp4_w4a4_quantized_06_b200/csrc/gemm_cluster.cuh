@@ -36,6 +36,17 @@
 
 namespace nvfp4 {
 
+// GDN gate activations of the a and b gate projections (ta-paperlens page,
+// "前提2"): a goes through softplus and the exponential, alpha = exp(-softplus(a))
+// (the share of the state that is kept), b through the logistic sigmoid,
+// beta = 1 / (1 + exp(-b)).  The model's per-head decay scale and bias are
+// not part of this layer (unit scale, zero bias).  CUDA's expf / log1pf.
+__device__ __forceinline__ float gate_keep(float a) {
+  const float sp = a > 0.0f ? a + log1pf(expf(-a)) : log1pf(expf(a));
+  return expf(-sp);
+}
+__device__ __forceinline__ float gate_write(float b) { return 1.0f / (1.0f + expf(-b)); }
+
 template <int BN>
 struct ClusterCfg {
   static constexpr int BM = 128;
@@ -317,8 +328,16 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
           if (s2 < S) acc = acc + red[s2 * slot + off];
         const float v = __fmul_rn(acc, alpha);
         const int64_t o = (int64_t)gi * p.out_si + (int64_t)gj * p.out_sj;
-        if constexpr (MODE == OUT_BF16) static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(v);
-        else static_cast<float *>(p.out)[o] = v;
+        if constexpr (MODE == OUT_BF16) {
+          static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(v);
+        } else if constexpr (MODE == OUT_GATES) {
+          // output column n is the weight row: tile row i for decode-shaped
+          // products, tile column j otherwise
+          const int n = i_fast ? gi : gj;
+          static_cast<float *>(p.out)[o] = n < p.n_split ? gate_keep(v) : gate_write(v);
+        } else {
+          static_cast<float *>(p.out)[o] = v;
+        }
       }
     }
   }

@@ -74,6 +74,7 @@ cudaError_t set_cluster_attrs() {
   const int b = ClusterCfg<BN>::SMEM_BYTES;
   cudaError_t e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, b);
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32>, b);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_GATES>, b);
   return e;
 }
 
@@ -336,17 +337,32 @@ nvfp4_status launch_gemm_bn(const CUtensorMap &ma, const CUtensorMap &mb, const 
   return launched();
 }
 
+template <int BN>
+cudaError_t launch_cluster(int mode, unsigned grid, int splits, bool pdl, const CUtensorMap &ma,
+                           const CUtensorMap &mb, const GemmParams &p, cudaStream_t stream) {
+  using C = ClusterCfg<BN>;
+  if (mode == OUT_BF16)
+    return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, grid, C::THREADS, C::SMEM_BYTES, stream, splits, pdl,
+                     ma, mb, p);
+  if (mode == OUT_GATES)
+    return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_GATES>, grid, C::THREADS, C::SMEM_BYTES, stream, splits, pdl,
+                     ma, mb, p);
+  return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_F32>, grid, C::THREADS, C::SMEM_BYTES, stream, splits, pdl,
+                   ma, mb, p);
+}
+
 // `pdl`: launched right after this library's activation quantize, which
 // lets the GEMM start early and stream the weight while the quantize ends.
 nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_gscale,
                        const uint8_t *b_codes, const uint8_t *b_sf, const float *b_gscale, void *y,
                        nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K, void *ws,
-                       size_t ws_bytes, cudaStream_t stream, bool pdl) {
+                       size_t ws_bytes, cudaStream_t stream, bool pdl, int64_t gates_n_a = -1) {
   DeviceState *dev = nullptr;
   nvfp4_status st = device_state(&dev);
   if (st != NVFP4_OK) return st;
   if (M == 0 || N == 0) return NVFP4_OK;
   const Plan pl = make_plan(M, N, K, *dev);
+  if (gates_n_a >= 0 && pl.kind != Plan::CLUSTER) return NVFP4_ERR_UNSUPPORTED;
   const size_t need = gemm_partial_bytes(M, N, K, *dev);
   if (need > 0 && (ws == nullptr || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
   if (need > 0 && !aligned16(ws)) return NVFP4_ERR_ALIGN;
@@ -415,28 +431,14 @@ nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float 
     CUtensorMap ma, mb;
     if (!make_codes_map(&ma, op_a, p.rows_a, K, 128) || !make_codes_map(&mb, op_b, p.rows_b, K, pl.bn))
       return NVFP4_ERR_CUDA;
-    cudaError_t e = cudaSuccess;
-    const bool bf = y_dt == NVFP4_OUT_BF16;
+    p.n_split = (int)(gates_n_a >= 0 ? gates_n_a : 0);
+    const int mode = gates_n_a >= 0 ? OUT_GATES : (y_dt == NVFP4_OUT_BF16 ? OUT_BF16 : OUT_F32);
     const unsigned g = (unsigned)pl.grid;
+    cudaError_t e;
     switch (pl.bn) {
-      case 32:
-        e = bf ? launch_ex(nvfp4_gemm_cluster_kernel<32, OUT_BF16>, g, ClusterCfg<32>::THREADS,
-                           ClusterCfg<32>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p)
-               : launch_ex(nvfp4_gemm_cluster_kernel<32, OUT_F32>, g, ClusterCfg<32>::THREADS,
-                           ClusterCfg<32>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p);
-        break;
-      case 64:
-        e = bf ? launch_ex(nvfp4_gemm_cluster_kernel<64, OUT_BF16>, g, ClusterCfg<64>::THREADS,
-                           ClusterCfg<64>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p)
-               : launch_ex(nvfp4_gemm_cluster_kernel<64, OUT_F32>, g, ClusterCfg<64>::THREADS,
-                           ClusterCfg<64>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p);
-        break;
-      default:
-        e = bf ? launch_ex(nvfp4_gemm_cluster_kernel<128, OUT_BF16>, g, ClusterCfg<128>::THREADS,
-                           ClusterCfg<128>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p)
-               : launch_ex(nvfp4_gemm_cluster_kernel<128, OUT_F32>, g, ClusterCfg<128>::THREADS,
-                           ClusterCfg<128>::SMEM_BYTES, stream, pl.splits, pdl, ma, mb, p);
-        break;
+      case 32: e = launch_cluster<32>(mode, g, pl.splits, pdl, ma, mb, p, stream); break;
+      case 64: e = launch_cluster<64>(mode, g, pl.splits, pdl, ma, mb, p, stream); break;
+      default: e = launch_cluster<128>(mode, g, pl.splits, pdl, ma, mb, p, stream); break;
     }
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     return launched();
@@ -730,6 +732,90 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
   if (w4a4_gemm_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return NVFP4_ERR_SCRATCH_LIMIT;
   return w4a4_gemm(x, x_dt, ld_x, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K, buf,
                    kNoAllocScratchBytes, stream);
+}
+
+nvfp4_status w4a4_gdn_gates(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                            const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, float *gates,
+                            int64_t ld_g, int64_t M, int64_t N, int64_t n_a, int64_t K, void *workspace,
+                            size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (x_dt != NVFP4_IN_BF16 && x_dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ld_x < K || n_a < 0 || n_a > N) return NVFP4_ERR_SHAPE;
+  if (N > 128) return NVFP4_ERR_UNSUPPORTED;        // the gate projections are narrow (N = 2 x heads)
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!x || !x_gscale) return NVFP4_ERR_NULL;
+  const int esz = x_dt == NVFP4_IN_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+  if (!workspace) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return NVFP4_ERR_ALIGN;
+  const size_t codes_b = align256(nvfp4_codes_bytes(M, K));
+  const size_t sf_b = align256(nvfp4_sf_bytes(M, K));
+  if (workspace_bytes < codes_b + sf_b) return NVFP4_ERR_WORKSPACE;
+  uint8_t *a_codes = static_cast<uint8_t *>(workspace);
+  uint8_t *a_sf = a_codes + codes_b;
+  nvfp4_status st = check_gemm_args(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, gates, NVFP4_OUT_F32, ld_g,
+                                    M, N, K);
+  if (st != NVFP4_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = quantize_impl(x, x_dt, M, K, ld_x, x_gscale, a_codes, a_sf, 0, M, s, true);
+  if (st != NVFP4_OK) return st;
+  return gemm_impl(a_codes, a_sf, x_gscale, w_codes, w_sf, w_gscale, gates, NVFP4_OUT_F32, ld_g, M, N, K,
+                   a_sf + sf_b, workspace_bytes - codes_b - sf_b, s, true, n_a);
+}
+
+nvfp4_status nvfp4_fake_quant(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                              const float *gscale, void *out, nvfp4_out_dtype out_dt, int64_t ld_out,
+                              double *err_stats, nvfp4_stream_t stream) {
+  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (out_dt != NVFP4_OUT_BF16 && out_dt != NVFP4_OUT_F32) return NVFP4_ERR_DTYPE;
+  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || ld_out < K || rows * ((K + 511) / 512) >= (int64_t)UINT32_MAX)
+    return NVFP4_ERR_SHAPE;
+  if (!gscale || (rows > 0 && (!x || !out))) return NVFP4_ERR_NULL;
+  const int esz = dt == NVFP4_IN_BF16 ? 2 : 4, osz = out_dt == NVFP4_OUT_BF16 ? 2 : 4;
+  if ((rows > 0 && (!aligned16(x) || !aligned16(out))) || (ld_x * esz) % 16 != 0 || (ld_out * osz) % 16 != 0 ||
+      (err_stats && (reinterpret_cast<uintptr_t>(err_stats) & 7)))
+    return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (err_stats && cudaMemsetAsync(err_stats, 0, 2 * sizeof(double), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (rows == 0) return NVFP4_OK;
+  FakeQuantParams p{x, rows, K, ld_x, gscale, out, ld_out, err_stats};
+  const int64_t units = rows * ((K + 511) / 512);
+  int64_t blocks = (units + 7) / 8;
+  if (blocks > 16LL * dev->sms) blocks = 16LL * dev->sms;
+  const unsigned g = (unsigned)blocks;
+  cudaError_t e;
+  if (dt == NVFP4_IN_BF16)
+    e = out_dt == NVFP4_OUT_F32 ? launch_ex(fake_quant_kernel<__nv_bfloat16, float>, g, 256u, 0, s, 0, false, p)
+                                : launch_ex(fake_quant_kernel<__nv_bfloat16, __nv_bfloat16>, g, 256u, 0, s, 0, false, p);
+  else
+    e = out_dt == NVFP4_OUT_F32 ? launch_ex(fake_quant_kernel<float, float>, g, 256u, 0, s, 0, false, p)
+                                : launch_ex(fake_quant_kernel<float, __nv_bfloat16>, g, 256u, 0, s, 0, false, p);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return launched();
+}
+
+nvfp4_status nvfp4_fp8_quantize(const void *x, nvfp4_in_dtype dt, int64_t n, const float *scale, uint8_t *q,
+                                nvfp4_stream_t stream) {
+  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (n < 0 || n % 8 != 0) return NVFP4_ERR_SHAPE;
+  if (n == 0) return NVFP4_OK;
+  if (!x || !scale || !q) return NVFP4_ERR_NULL;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7) || (reinterpret_cast<uintptr_t>(scale) & 3))
+    return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Fp8Params p{x, n, scale, q};
+  int64_t blocks = (n / 8 + 255) / 256;
+  if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
+  const cudaError_t e = dt == NVFP4_IN_BF16
+                            ? launch_ex(fp8_quantize_kernel<__nv_bfloat16>, (unsigned)blocks, 256u, 0, s, 0, false, p)
+                            : launch_ex(fp8_quantize_kernel<float>, (unsigned)blocks, 256u, 0, s, 0, false, p);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return launched();
 }
 
 nvfp4_status nvfp4_last_device_status(int *flags) {

@@ -468,6 +468,165 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   }
 }
 
+// ------------------------------------------------------ fake-quant (Q -> DQ)
+// Value of an E2M1 code: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6, sign in bit 3.
+__device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const uint32_t bits = m >= 2u ? ((126u + (m >> 1)) << 23) | ((m & 1u) << 22) : (m == 1u ? 0x3F000000u : 0u);
+  return __uint_as_float(bits | ((c & 8u) << 28));
+}
+
+struct FakeQuantParams {
+  const void *x;
+  int64_t rows, K, ld_x;
+  const float *gscale;
+  void *out;
+  int64_t ld_out;
+  double *stats;     // [sum of squared error, sum of squared input], or null
+};
+
+template <typename OUT>
+__device__ __forceinline__ void store16(OUT *dst, const float (&v)[16]);
+template <>
+__device__ __forceinline__ void store16<float>(float *dst, const float (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) reinterpret_cast<float4 *>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <>
+__device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[16]) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t *>(&h);
+  }
+  reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// Every element replaced by the NVFP4 value it quantizes to (the same
+// encoder as the quantize kernels, then dec(q) * dec(s) * g: the first
+// product is exact, so the result is fl32 of the exact value), plus the
+// float64 sums of the squared error against the exact value and of the
+// squared input.  One warp per 512-column
+// row segment, lane l owning block l, like quantize_rows_kernel.
+template <typename T, typename OUT>
+__global__ void __launch_bounds__(256) fake_quant_kernel(FakeQuantParams p) {
+  __shared__ float rcp_tab[128];
+  fill_rcp_table(rcp_tab);
+  pdl_prologue();
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t nseg = (uint32_t)((p.K + 511) >> 9);
+  const uint32_t units = (uint32_t)p.rows * nseg;
+  const EncodeConsts kc = encode_consts(p.gscale);
+  const T *x = static_cast<const T *>(p.x);
+  OUT *out = static_cast<OUT *>(p.out);
+  double se = 0.0, sx = 0.0;
+  for (uint32_t u = warp; u < units; u += nwarps) {
+    const int64_t row = u / nseg;
+    const int col = (int)(u - (uint32_t)row * nseg) * 512 + lane * 16;
+    if (col >= p.K) continue;
+    const T *src = x + row * p.ld_x + col;
+    Block16<T> b;
+    b.load(src);
+    uint32_t s;
+    const uint2 w = encode16(b, kc, rcp_tab, src, &s);
+    const float ds = e4m3_to_f32(s);
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t c = ((e < 8 ? w.x : w.y) >> ((e & 7) * 4)) & 0xFu;
+      const float qs = __fmul_rn(e2m1_to_f32(c), ds);            // exact: at most 7 significant bits
+      v[e] = __fmul_rn(qs, kc.g);
+      // the error is taken against the exact NVFP4 value (exact in float64)
+      const double xe = (double)b.elem(e), d = xe - (double)qs * (double)kc.g;
+      se = fma(d, d, se);
+      sx = fma(xe, xe, sx);
+    }
+    store16<OUT>(out + row * p.ld_out + col, v);
+  }
+  if (p.stats) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      se += __shfl_xor_sync(0xFFFFFFFFu, se, o);
+      sx += __shfl_xor_sync(0xFFFFFFFFu, sx, o);
+    }
+    if (lane == 0) {
+      atomicAdd(p.stats, se);
+      atomicAdd(p.stats + 1, sx);
+    }
+  }
+}
+
+// ------------------------------------------------- FP8 (E4M3) KV quantize
+// q = E4M3_RNE_SATFINITE(fl32(x / s)) with a static per-tensor scale s (sign
+// in bit 7).  Decided like the block scales: x * fl32(1/s) widened by 2^-21
+// both ways brackets fl32(x/s); equal hardware conversions are the answer,
+// otherwise the two neighbouring codes' midpoint is compared exactly.
+struct Fp8Params {
+  const void *x;
+  int64_t n;            // elements, a multiple of 8
+  const float *scale;
+  uint8_t *q;
+};
+
+__device__ __forceinline__ uint32_t fp8_settle(float x, float s, uint32_t lo, uint32_t hi) {
+  const uint32_t ml = lo & 0x7Fu, mh = hi & 0x7Fu;
+  const uint32_t m0 = min(ml, mh), m1 = max(ml, mh);
+  const float mid = __fmul_rn(__fadd_rn(e4m3_to_f32(m0), e4m3_to_f32(m1)), 0.5f);
+  const int c = quotient_vs(fabsf(x), s, mid);
+  const uint32_t m = c > 0 ? m1 : (c < 0 ? m0 : ((m0 & 1u) ? m1 : m0));
+  return m | (__float_as_uint(x) >> 24 & 0x80u);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) fp8_quantize_kernel(Fp8Params p) {
+  pdl_prologue();
+  const float s = __ldg(p.scale);
+  const bool fast = s >= 8.67361738e-19f && s <= 1.15292150e18f;   // 2^-60 .. 2^60
+  const float rs = __frcp_rn(s);
+  const float rlo = __fmul_rn(rs, kWidenLo), rhi = __fmul_rn(rs, kWidenHi);
+  const T *x = static_cast<const T *>(p.x);
+  const int64_t chunks = p.n >> 3;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float v[8];
+    if constexpr (sizeof(T) == 2) {
+      const uint4 r = __ldg(reinterpret_cast<const uint4 *>(x) + i);
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] = __uint_as_float(w[k] << 16);
+        v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    } else {
+      const float4 a = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
+      const float4 b = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t code;
+      if (fast) {
+        uint16_t pr;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(__fmul_rn(v[k], rhi)), "f"(__fmul_rn(v[k], rlo)));
+        const uint32_t lo = pr & 0xFFu, hi = (uint32_t)(pr >> 8);
+        code = lo == hi ? lo : fp8_settle(v[k], s, lo, hi);
+      } else {
+        uint16_t pr;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(0.0f), "f"(div_rn_slow(v[k], s)));
+        code = pr & 0xFFu;
+      }
+      out[k >> 2] |= code << ((k & 3) * 8);
+    }
+    reinterpret_cast<uint2 *>(p.q)[i] = make_uint2(out[0], out[1]);
+  }
+}
+
 // ------------------------------------------------------------- global scale
 template <typename T>
 __global__ void __launch_bounds__(256) amax_kernel(const T *x, int64_t rows, int64_t K, int64_t ld,

@@ -47,11 +47,15 @@ def lib() -> ctypes.CDLL:
         L.w4a4_gemm_workspace_bytes.argtypes, L.w4a4_gemm_workspace_bytes.restype = [i64, i64, i64], sz
         L.w4a4_gemm.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, sz, vp]
         L.w4a4_gemm_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp]
+        L.w4a4_gdn_gates.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, sz, vp]
+        L.nvfp4_fake_quant.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, i64, vp, vp]
+        L.nvfp4_fp8_quantize.argtypes = [vp, i32, i64, vp, vp, vp]
         L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
-                  "w4a4_gemm", "w4a4_gemm_noalloc", "nvfp4_last_device_status"):
+                  "w4a4_gemm", "w4a4_gemm_noalloc", "w4a4_gdn_gates", "nvfp4_fake_quant", "nvfp4_fp8_quantize",
+                  "nvfp4_last_device_status"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -191,6 +195,50 @@ def linear_noalloc(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tenso
     _check("w4a4_gemm_noalloc", lib().w4a4_gemm_noalloc(
         _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
         _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _stream()))
+    return out
+
+
+def gdn_gates(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
+              w_gscale: torch.Tensor, n_a: int, out: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The fused GDN gate projection: [M, N] float32 with alpha = exp(-softplus(a))
+    in columns [0, n_a) and beta = sigmoid(b) in the rest."""
+    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=x.device)
+    _check("w4a4_gdn_gates", lib().w4a4_gdn_gates(
+        _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
+        _ptr(out), out.stride(0), M, N, int(n_a), K, _ptr(workspace), workspace.numel(), _stream()))
+    return out
+
+
+def fake_quant(x: torch.Tensor, gscale: torch.Tensor, out_dtype=torch.float32,
+               stats: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Quantize-then-dequantize x; returns (values, [sum sq error, sum sq x] float64)."""
+    _require_cuda(x, gscale)
+    rows, K = x.shape
+    out = torch.empty((rows, K), dtype=out_dtype, device=x.device)
+    if stats is None:
+        stats = torch.empty(2, dtype=torch.float64, device=x.device)
+    _check("nvfp4_fake_quant", lib().nvfp4_fake_quant(
+        _ptr(x), _in_dtype(x), rows, K, x.stride(0), _ptr(gscale), _ptr(out), _out_dtype(out_dtype),
+        out.stride(0), _ptr(stats), _stream()))
+    return out, stats
+
+
+def fp8_quantize(x: torch.Tensor, scale: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """FP8 E4M3 codes (uint8, sign in bit 7) of x / scale, x contiguous."""
+    _require_cuda(x, scale)
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check("nvfp4_fp8_quantize", lib().nvfp4_fp8_quantize(_ptr(x), _in_dtype(x), x.numel(), _ptr(scale),
+                                                          _ptr(out), _stream()))
     return out
 
 

@@ -92,3 +92,24 @@ def test_empty_inputs_are_no_ops(L):
     assert L.nvfp4_quantize(None, 0, 0, 64, 64, None, None, None, 0, 0, None) == 0
     assert L.nvfp4_gemm(*([None] * 7), 0, 8, 0, 8, 64, None, 0, None) == 0
     assert L.w4a4_gemm(None, 0, 64, None, None, None, None, None, 0, 8, 0, 8, 64, None, 0, None) == 0
+
+
+def test_next_rows_validation(L):
+    g = L.w4a4_gdn_gates
+    base = [FAKE, 0, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 96]
+    assert g(*base, 64, 96, 48, 256, FAKE, 1 << 30, None) != 2              # well-formed up to here
+    assert g(*base, 64, 200, 48, 256, FAKE, 1 << 30, None) == 5             # N > 128: not a gate projection
+    assert g(*base, 64, 96, 97, 256, FAKE, 1 << 30, None) == 2              # n_a beyond N
+    assert g(*base, 64, 96, 48, 100, FAKE, 1 << 30, None) == 2              # K % 64
+    assert g(FAKE, 7, 256, FAKE, FAKE, FAKE, FAKE, FAKE, 96, 64, 96, 48, 256, FAKE, 1 << 30, None) == 4
+    f = L.nvfp4_fake_quant
+    assert f(FAKE, 0, 4, 100, 100, FAKE, FAKE, 1, 100, None, None) == 2      # K % 64
+    assert f(FAKE, 0, 4, 64, 64, FAKE, FAKE, 9, 64, None, None) == 4         # output dtype
+    assert f(FAKE + 2, 0, 4, 64, 64, FAKE, FAKE, 1, 64, None, None) == 3     # misaligned x
+    assert f(FAKE, 0, 4, 64, 64, FAKE, FAKE, 1, 64, FAKE + 4, None) == 3     # misaligned statistics
+    q = L.nvfp4_fp8_quantize
+    assert q(FAKE, 0, 12, FAKE, FAKE, None) == 2                             # n % 8
+    assert q(FAKE, 3, 16, FAKE, FAKE, None) == 4
+    assert q(FAKE, 0, 16, None, FAKE, None) == 1
+    assert q(FAKE + 8, 0, 16, FAKE, FAKE, None) == 3
+    assert q(FAKE, 0, 0, None, None, None) == 0                              # empty: nothing to do
