@@ -525,13 +525,26 @@ __global__ void __launch_bounds__(256) fake_quant_kernel(FakeQuantParams p) {
   const T *x = static_cast<const T *>(p.x);
   OUT *out = static_cast<OUT *>(p.out);
   double se = 0.0, sx = 0.0;
-  for (uint32_t u = warp; u < units; u += nwarps) {
-    const int64_t row = u / nseg;
-    const int col = (int)(u - (uint32_t)row * nseg) * 512 + lane * 16;
-    if (col >= p.K) continue;
+  for (uint32_t u0 = warp * 2; u0 < units; u0 += nwarps * 2) {
+    // two row segments per warp: both loads in flight before either is encoded
+    Block16<T> bb[2];
+    int64_t rr[2];
+    int cc[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t u = u0 + h;
+      rr[h] = u / nseg;
+      cc[h] = (int)(u - (uint32_t)rr[h] * nseg) * 512 + lane * 16;
+      bb[h].zero();
+      if (u < units && cc[h] < p.K) bb[h].load(x + rr[h] * p.ld_x + cc[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+    if (u0 + h >= units || cc[h] >= p.K) continue;
+    const int64_t row = rr[h];
+    const int col = cc[h];
     const T *src = x + row * p.ld_x + col;
-    Block16<T> b;
-    b.load(src);
+    const Block16<T> &b = bb[h];
     uint32_t s;
     const uint2 w = encode16(b, kc, rcp_tab, src, &s);
     const float ds = e4m3_to_f32(s);
@@ -547,6 +560,7 @@ __global__ void __launch_bounds__(256) fake_quant_kernel(FakeQuantParams p) {
       sx = fma(xe, xe, sx);
     }
     store16<OUT>(out + row * p.ld_out + col, v);
+    }
   }
   if (p.stats) {
 #pragma unroll
@@ -591,39 +605,56 @@ __global__ void __launch_bounds__(256) fp8_quantize_kernel(Fp8Params p) {
   const float rlo = __fmul_rn(rs, kWidenLo), rhi = __fmul_rn(rs, kWidenHi);
   const T *x = static_cast<const T *>(p.x);
   const int64_t chunks = p.n >> 3;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float v[8];
-    if constexpr (sizeof(T) == 2) {
-      const uint4 r = __ldg(reinterpret_cast<const uint4 *>(x) + i);
-      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  constexpr int U = 4;      // chunks loaded before any is converted
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < chunks;
+       base += U * nthreads) {
+    float v[U][8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[2 * k] = __uint_as_float(w[k] << 16);
-        v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    for (int c = 0; c < U; ++c) {
+      const int64_t i = base + c * nthreads;
+      if (i >= chunks) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[c][k] = 0.0f;
+        continue;
       }
-    } else {
-      const float4 a = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
-      const float4 b = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-    uint32_t out[2] = {0u, 0u};
+      if constexpr (sizeof(T) == 2) {
+        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(x) + i);
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint32_t code;
-      if (fast) {
-        uint16_t pr;
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(__fmul_rn(v[k], rhi)), "f"(__fmul_rn(v[k], rlo)));
-        const uint32_t lo = pr & 0xFFu, hi = (uint32_t)(pr >> 8);
-        code = lo == hi ? lo : fp8_settle(v[k], s, lo, hi);
+        for (int k = 0; k < 4; ++k) {
+          v[c][2 * k] = __uint_as_float(w[k] << 16);
+          v[c][2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        }
       } else {
-        uint16_t pr;
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(0.0f), "f"(div_rn_slow(v[k], s)));
-        code = pr & 0xFFu;
+        const float4 a4 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
+        const float4 b4 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
+        v[c][0] = a4.x; v[c][1] = a4.y; v[c][2] = a4.z; v[c][3] = a4.w;
+        v[c][4] = b4.x; v[c][5] = b4.y; v[c][6] = b4.z; v[c][7] = b4.w;
       }
-      out[k >> 2] |= code << ((k & 3) * 8);
     }
-    reinterpret_cast<uint2 *>(p.q)[i] = make_uint2(out[0], out[1]);
+#pragma unroll
+    for (int c = 0; c < U; ++c) {
+      const int64_t i = base + c * nthreads;
+      if (i >= chunks) continue;
+      uint32_t out[2] = {0u, 0u};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint32_t code;
+        if (fast) {
+          uint16_t pr;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(__fmul_rn(v[c][k], rhi)), "f"(__fmul_rn(v[c][k], rlo)));
+          const uint32_t lo = pr & 0xFFu, hi = (uint32_t)(pr >> 8);
+          code = lo == hi ? lo : fp8_settle(v[c][k], s, lo, hi);
+        } else {
+          uint16_t pr;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(0.0f), "f"(div_rn_slow(v[c][k], s)));
+          code = pr & 0xFFu;
+        }
+        out[k >> 2] |= code << ((k & 3) * 8);
+      }
+      reinterpret_cast<uint2 *>(p.q)[i] = make_uint2(out[0], out[1]);
+    }
   }
 }
 
