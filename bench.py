@@ -96,6 +96,22 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- helpers
+def max_over_ranks(values, world: int, device):
+    """Elementwise maximum of per-rank timings (the slowest replica sets the
+    job's time); a no-op on one rank."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(work_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job rate: every replica processes work_per_rank units in the
+    (max-over-ranks) time ms; returns units per second / 1e12."""
+    return work_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def quantized_weight(wl, dev):
     """Offline weight preparation: per-module quantize into the fused buffer,
     then the fused-group global-scale harmonization (untimed)."""
@@ -195,15 +211,10 @@ def run_native(args, rank, world, dev):
     total_ms = t_start.elapsed_time(t_end)
     tq = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
     tg = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
-    if world > 1:
-        t = torch.tensor([total_ms, sum(tq), sum(tg)], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, sq, sg = t.tolist()
-    else:
-        sq, sg = sum(tq), sum(tg)
+    total_ms, sq, sg = max_over_ranks([total_ms, sum(tq), sum(tg)], world, dev)
     ms_per_step = total_ms / args.steps
     flops = 2.0 * M * N * K
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(flops, world, ms_per_step)
     pk = peaks()
     tq_ms, tg_ms = sq / args.steps, sg / args.steps
     # the GEMM runs back to back for the whole timed region (a second or more
@@ -284,12 +295,9 @@ def measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world, steps
     e1.record(s)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks([ms], world, dev)[0]
     del ws, x_dev, y_dev
-    return {"value": round(2.0 * M * N * K * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    return {"value": round(job_throughput(2.0 * M * N * K, world, ms), 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": x_host.numel() * 2,
             "d2h_bytes_per_step": y_host.numel() * 2}
 
