@@ -367,6 +367,21 @@ def measure_secondary(native, dev):
                      "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
                      "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
                      "l2": f"CUDA graph over {copies} weight copies ({copies * wbytes / 1e6:.0f} MB)"}
+        # the same calls through the one-kernel variant (activation quantized in the GEMM)
+        gf = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gf):
+            for i in range(copies):
+                native.linear_fused(x, gx, wcs[i], wsfs[i], gw, out=y)
+        gf.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            gf.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        msf = e0.elapsed_time(e1) / (reps * copies)
+        res[name]["fused_prologue_us"] = round(msf * 1e3, 2)
+        del gf
         del g, wcs, wsfs, x, y, ws
     # rows beyond the layer: fused gate epilogue, fake-quant, FP8 KV quantize
     wl = W.WORKLOADS["gdn_gates_ab"]

@@ -217,6 +217,22 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
                                int64_t K, nvfp4_stream_t stream);
 
 /*
+ * The decode-shaped layer with the activation quantize inside the GEMM (row
+ * a9 of the layer, "quantize in the producer"): one kernel, whose extra warps
+ * encode each K stage of x straight into the MMA's operand tiles; the codes
+ * are bit-identical to nvfp4_quantize's and y is bit-identical to w4a4_gemm's.
+ * For M <= 128 activation rows only (NVFP4_ERR_UNSUPPORTED otherwise, and for
+ * shapes whose plan is not the narrow split-K one).  No workspace.  On B200
+ * this is slower than w4a4_gemm for the decode configurations (every weight
+ * tile's CTAs re-encode the same activation slice), so w4a4_gemm does not use
+ * it; it is kept as the in-producer variant of the layer.
+ */
+nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                             const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
+                             nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K,
+                             nvfp4_stream_t stream);
+
+/*
  * ------------------------------------------------------------------------
  * Rows beyond the layer itself, built on the same encoder and GEMM.
  * ------------------------------------------------------------------------

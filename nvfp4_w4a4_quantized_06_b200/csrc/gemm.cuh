@@ -48,6 +48,9 @@ struct GemmParams {
   int kstages;              // ceil(K / 256)
   int tiles_a, tiles_b, splits, group;
   int n_split;              // OUT_GATES: first output column of the b gates
+  const void *x;            // fused activation quantize: bf16/fp32 activation [rows_b, K]
+  int64_t ld_x;             //   its row stride (elements)
+  const float *x_gscale;    //   its global scale (device)
   unsigned *err;
 };
 

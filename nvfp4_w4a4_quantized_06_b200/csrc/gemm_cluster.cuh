@@ -31,8 +31,11 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include <type_traits>
+
 #include "gemm.cuh"
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace nvfp4 {
 
@@ -47,7 +50,11 @@ __device__ __forceinline__ float gate_keep(float a) {
 }
 __device__ __forceinline__ float gate_write(float b) { return 1.0f / (1.0f + expf(-b)); }
 
-template <int BN>
+// FUSED: the activation (the B operand of decode-shaped products) is read
+// as bf16/fp32 and quantized inside the kernel by QWARPS extra warps, which
+// write the codes straight into the MMA's swizzled B tiles and the scale
+// bytes into the B scale atoms ("quantize in the producer").
+template <int BN, bool FUSED = false>
 struct ClusterCfg {
   static constexpr int BM = 128;
   static constexpr int A_BYTES = BM * 128;                 // 256 FP4 per row per stage
@@ -58,7 +65,8 @@ struct ClusterCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = BN <= 32 ? 8 : (BN <= 64 ? 6 : 4);
   static constexpr int EPI_WARPS = 4;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int QWARPS = FUSED ? 8 : 0;
+  static constexpr int THREADS = 64 + 32 * (EPI_WARPS + QWARPS);
   static constexpr int SF_COLS = 16 + 16 * SFB_ATOMS;
   static constexpr int SFA_COL = BN;
   static constexpr int SFB_COL = BN + 16;
@@ -70,8 +78,9 @@ struct ClusterCfg {
   // of RED_PITCH floats (16-byte rows for vector stores); S*ceil(128/S) <= 135
   static constexpr int RED_PITCH = BN + 4;
   static constexpr int RED_FLOATS = ((BM + MAX_SPLITS - 1) * RED_PITCH + 31) / 32 * 32;   // 128-byte multiple
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RED_FLOATS * 4 + 256;
-  static_assert((3 * STAGES + 2) * 8 + 8 <= 256, "barrier area");
+  static constexpr int BAR_BYTES = 512;            // barriers, TMEM address, abort flag
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RED_FLOATS * 4 + BAR_BYTES + (FUSED ? 512 : 0);
+  static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier area");
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                     ((uint32_t)(BM >> 4) << 24);
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 128, "MMA N");
@@ -84,11 +93,15 @@ struct ClusterCfg {
 // p.splits = S (the cluster size), p.tiles_a x p.tiles_b tiles (one per
 // cluster), p.group != 0 when A is the operand independent of the preceding
 // kernel (the weight), 0 when B is.
-template <int BN, int MODE>
-__global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
+// XT = void: both operands pre-quantized (TMA); XT = bf16 / float: the B
+// operand is the activation p.x [rows_b, K] (row stride p.ld_x), quantized
+// here with global scale p.x_gscale (then tmb is unused).
+template <int BN, int MODE, typename XT = void>
+__global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THREADS, 1)
     nvfp4_gemm_cluster_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                               const GemmParams p) {
-  using C = ClusterCfg<BN>;
+  constexpr bool FUSED = !std::is_void<XT>::value;
+  using C = ClusterCfg<BN, FUSED>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -100,10 +113,12 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
   uint64_t *full = bars;
   uint64_t *empty = bars + C::STAGES;
   uint64_t *sfready = bars + 2 * C::STAGES;     // the stage's scales are in TMEM (4 warps)
-  uint64_t *tfull = bars + 3 * C::STAGES;
+  uint64_t *bready = bars + 3 * C::STAGES;      // FUSED: the stage's activation tile is encoded
+  uint64_t *tfull = bars + 4 * C::STAGES;
   uint64_t *tdone = tfull + 1;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tfull + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+  float *rcp_tab = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + C::BAR_BYTES);   // FUSED
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.splits;
@@ -121,6 +136,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sfready[s], C::EPI_WARPS);
+      if (FUSED) mbar_init(&bready[s], C::QWARPS);
     }
     mbar_init(tfull, 1);
     mbar_init(tdone, 1);
@@ -132,6 +148,12 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  if constexpr (FUSED) {
+    fill_rcp_table(rcp_tab);
+    // scale atoms of B rows past BN stay zero for the whole kernel
+    for (int i = threadIdx.x; i < C::STAGES * C::SFB_BYTES / 16; i += C::THREADS)
+      reinterpret_cast<uint4 *>(sSFB)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   tc_fence_before();
   __syncthreads();
@@ -153,6 +175,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
 #pragma unroll
         for (int j = 0; j < C::SFB_ATOMS; ++j)
           if (row_b + 128 * j < pad_b) ++nsfb;
+        if (FUSED) return (uint32_t)C::A_BYTES + (uint32_t)nkb * 512u;
         return (uint32_t)(C::A_BYTES + C::B_BYTES) + (uint32_t)nkb * 512u * (1u + nsfb);
       };
       auto load_a = [&](int st, int ks) {
@@ -162,6 +185,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
                   nkb * 512u, &full[st]);
       };
       auto load_b = [&](int st, int ks) {
+        if (FUSED) return;
         const int nkb = min(4, p.kblocks - ks * 4);
         tma_load_2d(sB + st * C::B_BYTES, &tmb, &full[st], ks * 128, row_b);
 #pragma unroll
@@ -211,6 +235,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       bool ok = true;
       for (int ks = ks0; ks < ks1; ++ks) {
         if (!mbar_wait(&sfready[st], ph, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
+        if (FUSED && !mbar_wait(&bready[st], ph, p.err, ERR_MMA, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint64_t ad = a_desc0 + (uint64_t)((st * C::A_BYTES) >> 4);
         const uint64_t bd = b_desc0 + (uint64_t)((st * C::B_BYTES) >> 4);
@@ -231,6 +256,47 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       volatile int never = 0;
       mbar_wait(tdone, 0, p.err, ERR_MMA, &never);
     }
+  } else if (FUSED && warp >= 2 + C::EPI_WARPS) {
+    if constexpr (FUSED) {
+      // -------------------------------------------- activation encoder warps
+      // Per K stage, the BN x 256 activation slice is encoded (same encoder
+      // as the quantize kernels, bit-identical codes) into this stage's B tile
+      // in the MMA's 128-byte-swizzled K-major layout (row r, 16-byte chunk c
+      // at r*128 + (c ^ (r % 8))*16) and its scale bytes into the stage's B
+      // scale atoms.  Rows past rows_b and columns past K encode as zeros.
+      const int qt = (int)threadIdx.x - 32 * (2 + C::EPI_WARPS);
+      constexpr int QT = 32 * C::QWARPS;
+      griddep_wait();                                     // x and its scale may come from the preceding kernel
+      const EncodeConsts kc = encode_consts(p.x_gscale);
+      const XT *x = static_cast<const XT *>(p.x);
+      int st = 0;
+      uint32_t ph = 0;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        // the stage's previous tiles have been consumed by the MMAs
+        if (!mbar_wait_warp(&empty[st], ph ^ 1, p.err, ERR_PRODUCER, abort_flag)) break;
+        uint8_t *sb = sB + st * C::B_BYTES;
+        uint8_t *ssf = sSFB + st * C::SFB_BYTES;
+#pragma unroll 1
+        for (int bi = qt; bi < BN * 16; bi += QT) {
+          const int r = bi >> 4, b = bi & 15;
+          const int64_t col = (int64_t)ks * 256 + b * 16;
+          uint2 w = make_uint2(0u, 0u);
+          uint32_t sc = 0u;
+          if (r < p.rows_b && col < p.K) {
+            const XT *src = x + (int64_t)r * p.ld_x + col;
+            Block16<XT> blk;
+            blk.load(src);
+            w = encode16(blk, kc, rcp_tab, src, &sc);
+          }
+          *reinterpret_cast<uint2 *>(sb + r * 128 + (((b >> 1) ^ (r & 7)) << 4) + (b & 1) * 8) = w;
+          ssf[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)] = (uint8_t)sc;
+        }
+        fence_proxy_async_shared();                      // the tensor core reads the tile through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bready[st]);
+        if (++st == C::STAGES) { st = 0; ph ^= 1; }
+      }
+    }
   } else {
     const int q = warp & 3;                       // TMEM lane quarter of this warp
     const int i = q * 32 + lane;                  // tile row (A row)
@@ -246,6 +312,7 @@ __global__ void __launch_bounds__(ClusterCfg<BN>::THREADS, 1)
       uint32_t ph = 0;
       for (int ks = ks0; ks < ks1; ++ks) {
         if (!mbar_wait_warp(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
+        if (FUSED && !mbar_wait_warp(&bready[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
         const uint4 *sa = reinterpret_cast<const uint4 *>(sSFA + st * C::SFA_BYTES) + lane;
         const uint4 *sb = reinterpret_cast<const uint4 *>(sSFB + st * C::SFB_BYTES) + lane;
         const uint32_t reg = tmem + lane_addr + (uint32_t)(st * C::SF_COLS);

@@ -75,6 +75,11 @@ cudaError_t set_cluster_attrs() {
   cudaError_t e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, b);
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32>, b);
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_GATES>, b);
+  const int bf = ClusterCfg<BN, true>::SMEM_BYTES;
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_BF16, __nv_bfloat16>, bf);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32, __nv_bfloat16>, bf);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_BF16, float>, bf);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32, float>, bf);
   return e;
 }
 
@@ -349,6 +354,68 @@ cudaError_t launch_cluster(int mode, unsigned grid, int splits, bool pdl, const 
                      ma, mb, p);
   return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_F32>, grid, C::THREADS, C::SMEM_BYTES, stream, splits, pdl,
                    ma, mb, p);
+}
+
+template <int BN, typename XT>
+cudaError_t launch_cluster_fused(bool bf16_out, unsigned grid, int splits, const CUtensorMap &ma,
+                                 const GemmParams &p, cudaStream_t stream) {
+  using C = ClusterCfg<BN, true>;
+  return bf16_out ? launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_BF16, XT>, grid, C::THREADS, C::SMEM_BYTES, stream,
+                              splits, true, ma, ma, p)
+                  : launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_F32, XT>, grid, C::THREADS, C::SMEM_BYTES, stream,
+                              splits, true, ma, ma, p);
+}
+
+// The decode-shaped layer in one kernel: the activation x (M <= 128 rows)
+// is quantized inside the cluster GEMM (row a9).  Returns UNSUPPORTED when the
+// plan is not a cluster plan with the activation on the narrow side.
+nvfp4_status w4a4_fused_impl(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                             const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
+                             nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K,
+                             const DeviceState &dev, cudaStream_t stream) {
+  const Plan pl = make_plan(M, N, K, dev);
+  if (pl.kind != Plan::CLUSTER || !pl.swap) return NVFP4_ERR_UNSUPPORTED;
+  GemmParams p{};
+  p.sfa = w_sf;
+  p.ga = x_gscale;
+  p.gb = w_gscale;
+  p.rows_a = (int)N;
+  p.rows_b = (int)M;
+  p.K = (int)K;
+  p.kblocks = (int)(K / 64);
+  p.kstages = pl.kstages;
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.splits = pl.splits;
+  p.group = 1;
+  p.err = dev.err;
+  p.out = y;
+  p.out_si = 1;
+  p.out_sj = ld_y;
+  p.x = x;
+  p.ld_x = ld_x;
+  p.x_gscale = x_gscale;
+  CUtensorMap ma;
+  if (!make_codes_map(&ma, w_codes, N, K, 128)) return NVFP4_ERR_CUDA;
+  const bool bf = y_dt == NVFP4_OUT_BF16, xb = x_dt == NVFP4_IN_BF16;
+  const unsigned g = (unsigned)pl.grid;
+  cudaError_t e;
+  switch (pl.bn) {
+    case 32:
+      e = xb ? launch_cluster_fused<32, __nv_bfloat16>(bf, g, pl.splits, ma, p, stream)
+             : launch_cluster_fused<32, float>(bf, g, pl.splits, ma, p, stream);
+      break;
+    case 64:
+      e = xb ? launch_cluster_fused<64, __nv_bfloat16>(bf, g, pl.splits, ma, p, stream)
+             : launch_cluster_fused<64, float>(bf, g, pl.splits, ma, p, stream);
+      break;
+    default:
+      e = xb ? launch_cluster_fused<128, __nv_bfloat16>(bf, g, pl.splits, ma, p, stream)
+             : launch_cluster_fused<128, float>(bf, g, pl.splits, ma, p, stream);
+      break;
+  }
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return launched();
 }
 
 // `pdl`: launched right after this library's activation quantize, which
@@ -732,6 +799,26 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
   if (w4a4_gemm_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return NVFP4_ERR_SCRATCH_LIMIT;
   return w4a4_gemm(x, x_dt, ld_x, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K, buf,
                    kNoAllocScratchBytes, stream);
+}
+
+nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
+                             const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
+                             nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K,
+                             nvfp4_stream_t stream) {
+  if (x_dt != NVFP4_IN_BF16 && x_dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ld_x < K) return NVFP4_ERR_SHAPE;
+  if (M > 128) return NVFP4_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!x || !x_gscale) return NVFP4_ERR_NULL;
+  const int esz = x_dt == NVFP4_IN_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+  // the activation-side arguments stand in for the codes the kernel makes itself
+  nvfp4_status st = check_gemm_args(w_codes, w_sf, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K);
+  if (st != NVFP4_OK) return st;
+  DeviceState *dev = nullptr;
+  if ((st = device_state(&dev)) != NVFP4_OK) return st;
+  return w4a4_fused_impl(x, x_dt, ld_x, x_gscale, w_codes, w_sf, w_gscale, y, y_dt, ld_y, M, N, K, *dev,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status w4a4_gdn_gates(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,

@@ -329,6 +329,11 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (TMA stores, tcgen05.mma operand fetches)
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 // store a float into the shared memory of a CTA of this cluster (the
 // address from mapa); ordered before a later barrier.cluster.arrive.release
 __device__ __forceinline__ void st_shared_cluster_f32(uint32_t cluster_addr, float v) {

@@ -47,6 +47,7 @@ def lib() -> ctypes.CDLL:
         L.w4a4_gemm_workspace_bytes.argtypes, L.w4a4_gemm_workspace_bytes.restype = [i64, i64, i64], sz
         L.w4a4_gemm.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, sz, vp]
         L.w4a4_gemm_noalloc.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp]
+        L.w4a4_gemm_fused.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i32, i64, i64, i64, i64, vp]
         L.w4a4_gdn_gates.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, sz, vp]
         L.nvfp4_fake_quant.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, i64, vp, vp]
         L.nvfp4_fp8_quantize.argtypes = [vp, i32, i64, vp, vp, vp]
@@ -54,7 +55,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
-                  "w4a4_gemm", "w4a4_gemm_noalloc", "w4a4_gdn_gates", "nvfp4_fake_quant", "nvfp4_fp8_quantize",
+                  "w4a4_gemm", "w4a4_gemm_noalloc", "w4a4_gemm_fused", "w4a4_gdn_gates", "nvfp4_fake_quant", "nvfp4_fp8_quantize",
                   "nvfp4_last_device_status"):
             getattr(L, f).restype = i32
         _lib = L
@@ -193,6 +194,21 @@ def linear_noalloc(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tenso
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
     _check("w4a4_gemm_noalloc", lib().w4a4_gemm_noalloc(
+        _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
+        _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _stream()))
+    return out
+
+
+def linear_fused(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
+                 w_gscale: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """The decode-shaped layer (M <= 128) with the activation quantized inside
+    the GEMM kernel; bit-identical to linear()."""
+    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check("w4a4_gemm_fused", lib().w4a4_gemm_fused(
         _ptr(x), _in_dtype(x), x.stride(0), _ptr(x_gscale), _ptr(w_codes), _ptr(w_sf), _ptr(w_gscale),
         _ptr(out), _out_dtype(out.dtype), out.stride(0), M, N, K, _stream()))
     return out

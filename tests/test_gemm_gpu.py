@@ -173,3 +173,34 @@ def test_prefill_mlp_full_size():
     benchmark times, checked on a seeded sample of outputs."""
     wl = W.WORKLOADS["prefill_mlp_gate_up"]
     _run_linear(wl, torch.bfloat16, rows=W.sample_rows(wl.M, 64), cols=W.sample_rows(wl.N, 512, seed=9))
+
+
+@pytest.mark.parametrize("M,N,K,x_dtype", [
+    (1, 640, 2048, torch.bfloat16),
+    (32, 5120, 5120, torch.bfloat16),     # decode out_proj
+    (33, 1000, 1344, torch.float32),      # 64-wide MMA N, K tail, fp32 activation
+    (100, 2000, 1344, torch.bfloat16),    # 128-wide MMA N
+])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fused_prologue_matches_layer(M, N, K, x_dtype, out_dtype):
+    """The in-GEMM activation quantize gives the two-kernel layer's output bit
+    for bit (same codes, same MMAs, same reduction order)."""
+    x = W.gaussian(M, K, seed=M + 3, outliers=W.Outliers("scale", 0.02, 30.0), dtype=x_dtype).to(DEV)
+    w = W.gaussian(N, K, seed=N + 5, std=0.02).to(DEV)
+    gx, gw = native.amax_gscale(x), native.amax_gscale(w)
+    wc, ws = native.quantize(w, gw)
+    y_ref = native.linear(x, gx, wc, ws, gw, out_dtype=out_dtype)
+    y = native.linear_fused(x, gx, wc, ws, gw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+    assert torch.equal(y, y_ref)
+
+
+def test_fused_prologue_rejects_prefill_shapes():
+    x = torch.zeros(256, 256, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(256, 256, dtype=torch.bfloat16, device=DEV)
+    g = torch.ones(1, dtype=torch.float32, device=DEV)
+    wc, ws = native.quantize(w, g)
+    with pytest.raises(native.Nvfp4Error) as e:
+        native.linear_fused(x, g, wc, ws, g)
+    assert e.value.status == 5
