@@ -7,6 +7,12 @@
 // fl32(g_a * g_b) and writes BF16 or FP32, or writes raw FP32 partial sums for
 // a later split-K reduction.
 //
+// Used for the products the CTA-pair kernel (large M and N) and the cluster
+// split-K kernel (one operand of at most 128 rows) do not take: both
+// operands wider than 128 rows but too few 256 x 256 tiles to fill the
+// device with pairs.  This file also holds the parameter block, the tile
+// raster and the output helpers the other GEMM kernels share.
+//
 // Design (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: per K-stage of 256 elements, a 2D tiled load of
 //               the 128 x 128-byte A tile and the BN x 128-byte B tile (128-byte

@@ -1,6 +1,9 @@
 // quantize.cuh -- NVFP4 encoder kernels for sm_100a: per-tensor global scale,
-// activation/weight quantize (E2M1 codes + swizzled E4M3 block scales) and
-// fused-group global-scale harmonization.
+// activation/weight quantize (E2M1 codes + swizzled E4M3 block scales; a
+// TMA-fed streaming kernel and a generic per-row kernel), fused-group
+// global-scale harmonization, and the rows built on the same encoder:
+// fake-quant (quantize then dequantize, with error sums) and static-scale
+// FP8 E4M3 quantize.
 //
 // Format (web pages on arXiv 2609.04098; ta-paperlens page, section "前提1";
 // arxiv-wiki page, "접근 방법"): 4-bit E2M1 values, one E4M3 scale per 16
@@ -334,12 +337,19 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
     }
   }
   // zero the scale bytes of the padding rows this call owns
+  // (fewer than 128 rows of K/16 columns: 32-bit index arithmetic unless K is huge)
   const int64_t pad_bytes = p.pad_rows * ncols;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = tid; i < pad_bytes; i += nthreads) {
-    const int64_t r = p.sf_row0 + p.rows + i / ncols, c = i % ncols;
-    p.sf[sf_index(r, c, p.K)] = 0;
+  if (pad_bytes < (int64_t(1) << 31)) {
+    const uint32_t nc = (uint32_t)ncols;
+    for (uint32_t i = (uint32_t)tid; i < (uint32_t)pad_bytes; i += (uint32_t)nthreads) {
+      const uint32_t rr = i / nc, c = i - rr * nc;
+      p.sf[sf_index(p.sf_row0 + p.rows + rr, c, p.K)] = 0;
+    }
+  } else {
+    for (int64_t i = tid; i < pad_bytes; i += nthreads)
+      p.sf[sf_index(p.sf_row0 + p.rows + i / ncols, i % ncols, p.K)] = 0;
   }
 }
 
