@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -137,7 +138,12 @@ def kernel_src_hash():
     path must refresh profiles/dram_traffic.json by hand)."""
     h = hashlib.sha256()
     for f in ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh"):
-        h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_06_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "nvfp4_w4a4_quantized_06_b200", "csrc", f), encoding="utf-8").read()
+        # comments do not change the kernel: hash the code only
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        code = (line.split("//", 1)[0].rstrip() for line in text.splitlines())
+        text = "\n".join(line for line in code if line)
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 
