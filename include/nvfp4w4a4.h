@@ -233,6 +233,18 @@ nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, c
                              nvfp4_stream_t stream);
 
 /*
+ * Failure-detection self-test: launches one thread that waits, bounded by
+ * limit_ns of %globaltimer (0 < limit_ns <= 2e9), on a barrier nothing ever
+ * completes.  The wait runs out, sets bit 16 of the device error word (read
+ * and cleared by nvfp4_last_device_status, which then returns
+ * NVFP4_ERR_TIMEOUT) and writes 0 to *result_dev (device int); the kernel
+ * returns normally and the context stays usable.  Every wait in the library's
+ * kernels is bounded the same way (2 s), so a lost producer or consumer shows
+ * up as this status instead of a hang.
+ */
+nvfp4_status nvfp4_selftest_wait_timeout(int64_t limit_ns, int *result_dev, nvfp4_stream_t stream);
+
+/*
  * ------------------------------------------------------------------------
  * Rows beyond the layer itself, built on the same encoder and GEMM.
  * ------------------------------------------------------------------------

@@ -645,6 +645,35 @@ nvfp4_status quantize_impl(const void *x, nvfp4_in_dtype dt, int64_t rows, int64
                              : launch_quantize<float>(p, *dev, s, pdl);
 }
 
+constexpr unsigned ERR_SELFTEST = 16u;   // error-word bit of the self-test below
+
+// mbar_wait with a caller-chosen limit (the self-test of the timeout path).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, unsigned *err, unsigned code,
+                                                unsigned long long limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(a, parity)) return true;
+    if (globaltimer() - t0 > limit_ns) {
+      atomicOr(err, code);
+      return false;
+    }
+  }
+}
+
+// Failure-detection self-test: one thread waits on an mbarrier that nothing
+// arrives on, so the bounded wait runs out, records ERR_SELFTEST in the
+// error word and the kernel returns normally (no fault, no trap).
+__global__ void wait_timeout_selftest_kernel(unsigned *err, unsigned long long limit_ns, int *result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    const bool ok = mbar_wait_limit(&bar, 0, err, ERR_SELFTEST, limit_ns);
+    *result = ok ? 1 : 0;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -902,6 +931,17 @@ nvfp4_status nvfp4_fp8_quantize(const void *x, nvfp4_in_dtype dt, int64_t n, con
                             ? launch_ex(fp8_quantize_kernel<__nv_bfloat16>, (unsigned)blocks, 256u, 0, s, 0, false, p)
                             : launch_ex(fp8_quantize_kernel<float>, (unsigned)blocks, 256u, 0, s, 0, false, p);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return launched();
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(int64_t limit_ns, int *result_dev, nvfp4_stream_t stream) {
+  if (!result_dev) return NVFP4_ERR_NULL;
+  if (limit_ns <= 0 || limit_ns > 2000000000LL) return NVFP4_ERR_SHAPE;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      dev->err, (unsigned long long)limit_ns, result_dev);
   return launched();
 }
 

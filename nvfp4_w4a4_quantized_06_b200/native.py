@@ -51,12 +51,13 @@ def lib() -> ctypes.CDLL:
         L.w4a4_gdn_gates.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, sz, vp]
         L.nvfp4_fake_quant.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, i64, vp, vp]
         L.nvfp4_fp8_quantize.argtypes = [vp, i32, i64, vp, vp, vp]
+        L.nvfp4_selftest_wait_timeout.argtypes = [i64, vp, vp]
         L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
                   "w4a4_gemm", "w4a4_gemm_noalloc", "w4a4_gemm_fused", "w4a4_gdn_gates", "nvfp4_fake_quant", "nvfp4_fp8_quantize",
-                  "nvfp4_last_device_status"):
+                  "nvfp4_selftest_wait_timeout", "nvfp4_last_device_status"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -256,6 +257,14 @@ def fp8_quantize(x: torch.Tensor, scale: torch.Tensor, out: torch.Tensor | None 
     _check("nvfp4_fp8_quantize", lib().nvfp4_fp8_quantize(_ptr(x), _in_dtype(x), x.numel(), _ptr(scale),
                                                           _ptr(out), _stream()))
     return out
+
+
+def selftest_wait_timeout(limit_ns: int = 50_000_000) -> torch.Tensor:
+    """Run the bounded-wait self-test; returns the device int the waiter wrote
+    (0: the wait ran out, as intended)."""
+    res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check("nvfp4_selftest_wait_timeout", lib().nvfp4_selftest_wait_timeout(int(limit_ns), _ptr(res), _stream()))
+    return res
 
 
 def last_device_status() -> int:
