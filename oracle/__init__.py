@@ -14,15 +14,19 @@ repair on the arxiv-wiki page ("접근 방법", "개발자 관점") and the abst
 shd-paper page.  Readings the pages leave open are listed in the C file's
 header.  Everything except the arithmetic order for non-power-of-two global
 scales is pinned by tests/test_oracle_*.py; that order is "parity unpinned".
-The rows marked "next" (GDN gate activations, fake-quant, FP8 KV quantize)
-follow the same pages (ta-paperlens "前提2"; arxiv-wiki "주요 결과") and are
-pinned in tests/test_oracle_next.py.
+The rows marked "next" (GDN gate activations, fake-quant, FP8 KV quantize,
+the re-quantizing harmonize and the quantize fused into the preceding
+RMSNorm) follow the same pages (ta-paperlens "前提2": the GDN layer feeds the
+residual stream through its projections and every norm stays in BF16;
+arxiv-wiki "주요 결과", "접근 방법") and are pinned in tests/test_oracle_next.py.
 """
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
+from fractions import Fraction
 
 import numpy as np
 
@@ -208,6 +212,126 @@ def fp8_quantize(x: np.ndarray, s) -> np.ndarray:
     q = np.empty(x.shape, dtype=np.uint8)
     lib().oracle_fp8_quantize(_ptr(x), x.size, float(np.float32(s)), _ptr(q))
     return q
+
+
+def harmonize_requant(codes: np.ndarray, sf: np.ndarray, K: int, row_offsets, gscales):
+    """Re-quantizing harmonize of a fused group: every module's weights, taken
+    as their NVFP4 values rounded once to fp32 (the fake-quant value,
+    dec(q)*dec(s)*g_m), are quantized again against g* = max(g_m).  Codes and
+    scales both change.  Returns (codes', sf', g*); the inputs are not touched."""
+    offs = [int(o) for o in row_offsets]
+    gs = [np.float32(g) for g in gscales]
+    assert len(offs) == len(gs) + 1 and offs[0] == 0
+    gstar = max(gs)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out_codes = np.empty_like(codes)
+    out_sf = np.zeros_like(sf)
+    for m, g in enumerate(gs):
+        r0, r1 = offs[m], offs[m + 1]
+        xhat = dequantize(codes[r0:r1], sf, g, sf_row0=r0).astype(np.float32)   # one rounding of an exact value
+        out_codes[r0:r1], _ = quantize(xhat, gstar, sf=out_sf, sf_row0=r0)
+    return out_codes, out_sf, gstar
+
+
+# ---------------------------------------- quantize fused into RMSNorm
+RMS_NEAR_TIE = 2.0 ** -44   # |m^2 V - 1| below this: 1/sqrt(V) lies within ~2^-45 of an fp32 midpoint
+
+
+def _exact_sum_squares(row: np.ndarray) -> Fraction:
+    """Sum of x^2 over a row of float32 values, exactly: x = m * 2^(e-24) with
+    m an integer below 2^24, so x^2 = m^2 * 2^(2e-48); the m^2 of equal
+    exponents are added as integers and the groups shifted into one."""
+    mant, ex = np.frexp(row.astype(np.float64))
+    mi = np.ldexp(mant, 24).astype(np.int64)
+    assert np.array_equal(mi.astype(np.float64), np.ldexp(mant, 24)), "float32 input expected"
+    sq = mi * mi                                   # < 2^48, exact
+    e2 = 2 * (ex.astype(np.int64) - 24)
+    nz = mi != 0
+    if not np.any(nz):
+        return Fraction(0)
+    e0 = int(e2[nz].min())
+    total = 0
+    for k in np.unique(e2[nz]):
+        part = sq[nz & (e2 == k)]
+        s = (int((part >> 32).sum()) << 32) + int((part & 0xFFFFFFFF).sum())   # two halves: no int64 overflow
+        total += s << (int(k) - e0)
+    return Fraction(total) * Fraction(2) ** e0
+
+
+def rsqrt_rn32(V: Fraction):
+    """The float32 nearest to 1/sqrt(V) (ties to the even significand), for a
+    positive rational V, decided exactly: 1/sqrt(V) > m  <=>  m^2 V < 1 for a
+    midpoint m between neighbouring floats.  Also returns how close
+    1/sqrt(V) comes to either midpoint, as min |m^2 V - 1|."""
+    assert V > 0
+    f = np.float32(1.0 / math.sqrt(float(V)))
+    inf, zero = np.float32(np.inf), np.float32(0.0)
+    while True:
+        up, dn = np.nextafter(f, inf), np.nextafter(f, zero)
+        mh = (Fraction(float(f)) + Fraction(float(up))) / 2
+        ml = (Fraction(float(dn)) + Fraction(float(f))) / 2
+        th, tl = mh * mh * V, ml * ml * V
+        if th < 1:
+            f = up
+            continue
+        if tl > 1:
+            f = dn
+            continue
+        odd = int(np.array(f).view(np.uint32)) & 1
+        if th == 1 and odd:
+            f = up
+        elif tl == 1 and odd:
+            f = dn
+        return f, float(min(abs(th - 1), abs(tl - 1)))
+
+
+def rms_inv(x: np.ndarray, eps):
+    """Per row: inv = the float32 nearest to 1/sqrt(mean(x^2) + eps), with the
+    mean taken exactly (eps a positive float32), and whether the exact value
+    lies within ~2^-45 of a rounding midpoint (then a kernel that evaluates it
+    to ~2^-48 may round either way)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    e = Fraction(float(np.float32(eps)))
+    assert e > 0
+    rows, K = x.shape
+    inv = np.empty(rows, np.float32)
+    near = np.zeros(rows, bool)
+    for r in range(rows):
+        V = _exact_sum_squares(x[r]) / K + e
+        inv[r], close = rsqrt_rn32(V)
+        near[r] = close < RMS_NEAR_TIE
+    return inv, near
+
+
+def _bf16_rne(v: np.ndarray) -> np.ndarray:
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def rmsnorm(x: np.ndarray, w: np.ndarray, eps, zero_centered: bool = False, inv=None):
+    """RMSNorm of the residual stream as the BF16 input of the projections
+    that read it (the norms stay in BF16): h = fl32(x * inv),
+    y = bf16(fl32(h * gamma)) with gamma = w (or fl32(1 + w) for the
+    zero-centred form), w the norm weight (bf16 values).  Returns
+    (y as float32 [rows, K], inv [rows], near-tie flags [rows]); `inv`
+    overrides the per-row factor (for rows flagged near a tie)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    w = np.asarray(w, dtype=np.float32)
+    assert np.array_equal(_bf16_rne(w), w), "norm weight must hold bf16 values"
+    inv_rn, near = rms_inv(x, eps)
+    if inv is not None:
+        inv_rn = np.asarray(inv, dtype=np.float32)
+    h = x * inv_rn[:, None]                                   # float32 products, each rounded once
+    gamma = (np.float32(1.0) + w) if zero_centered else w
+    y = _bf16_rne(h * gamma[None, :])
+    return y, inv_rn, near
+
+
+def rmsnorm_quantize(x: np.ndarray, w: np.ndarray, eps, g, zero_centered: bool = False, inv=None):
+    """NVFP4 quantize of the RMSNorm output: (codes, sf, y, inv, near-tie)."""
+    y, inv_rn, near = rmsnorm(x, w, eps, zero_centered, inv)
+    codes, sf = quantize(y, g)
+    return codes, sf, y, inv_rn, near
 
 
 def num_threads() -> int:
