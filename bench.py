@@ -430,7 +430,40 @@ def measure_secondary(native, dev):
                               "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
                               "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
                               "rel_error": round(float(np.sqrt(st[0].item() / st[1].item())), 5)}
-    del x, fq
+    del fq
+    # quantize fused into the RMSNorm that produces this activation
+    wn = W.norm_weight(wl.K, seed=11).to(dev)
+    gy = native.amax_gscale(torch.nn.functional.rms_norm(x, (wl.K,), weight=wn, eps=1e-6))
+    yc = torch.empty((wl.M, wl.K // 2), dtype=torch.uint8, device=dev)
+    ysf = torch.empty(native.sf_bytes(wl.M, wl.K), dtype=torch.uint8, device=dev)
+    yinv = torch.empty(wl.M, dtype=torch.float32, device=dev)
+    ms = timed(lambda: native.rmsnorm_quantize(x, wn, 1e-6, gy, codes=yc, sf=ysf, inv=yinv))
+
+    def unfused():
+        y = torch.nn.functional.rms_norm(x, (wl.K,), weight=wn, eps=1e-6)
+        native.quantize(y, gy, codes=yc, sf=ysf)
+
+    ms_unfused = timed(unfused)
+    byts = wl.M * wl.K * 2 + wl.M * wl.K // 2 + wl.M * wl.K // 16 + wl.K * 2 + wl.M * 4
+    res["rmsnorm_quantize"] = {"shape": f"{wl.M}x{wl.K} bf16 residual", "ms": round(ms, 4),
+                               "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                               "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
+                               "unfused_torch_rms_norm_then_quantize_ms": round(ms_unfused, 4),
+                               "l2": "512 MB flush between reps"}
+    del x, yc, ysf, yinv
+    # re-quantizing harmonize of the fused qkv+z weight (offline; in place, so
+    # every rep re-encodes the previous rep's output)
+    wl = W.WORKLOADS["gdn_qkv_z"]
+    wc, wsf, gw = quantized_weight(wl, dev)
+    offs = [0, wl.modules[0], wl.N]
+    gsm = torch.cat([gw, gw * 0.8])
+    ms = timed(lambda: native.harmonize_requant(wc, wsf, wl.K, offs, gsm))
+    byts = 2 * (wl.N * wl.K // 2 + wl.N * wl.K // 16)
+    res["harmonize_requant_qkv_z"] = {"shape": f"{wl.N}x{wl.K}", "ms": round(ms, 4),
+                                      "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                                      "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
+                                      "l2": "512 MB flush between reps"}
+    del wc, wsf
     kv = torch.randn(32 * 4096 * 4 * 256 * 2, dtype=torch.bfloat16, device=dev)     # 32 seqs x 4096 tokens, K and V
     sc = (kv.abs().max().float() / 448.0).reshape(1)
     q8 = torch.empty(kv.numel(), dtype=torch.uint8, device=dev)

@@ -301,6 +301,54 @@ nvfp4_status nvfp4_fp8_quantize(const void *x, nvfp4_in_dtype dt, int64_t n, con
                                 nvfp4_stream_t stream);
 
 /*
+ * Re-quantizing variant of the fused-group repair (arxiv-wiki page,
+ * "접근 방법", last bullet: the modules of a fused GEMM must share one global
+ * scale).  Instead of rewriting only the scale bytes (nvfp4_harmonize_group),
+ * every block of module m is dequantized to fp32, v = fl32(dec(q) * dec(s) *
+ * g_m) (the fake-quant value), and encoded again against g* = max_m g_m with
+ * the same arithmetic as nvfp4_quantize.  Codes and scales both change where
+ * that moves them: wherever the new scale is a normal E4M3 value the codes
+ * come out unchanged and only the scale can differ from the scale-only
+ * rewrite; blocks pushed to subnormal scales get re-rounded codes.
+ *   codes, sf     : the fused group's codes [rows_total, K/2] and swizzled
+ *                   scales (device, both rewritten in place; padding rows
+ *                   untouched).
+ *   row_offsets, gscales, shared_gscale_out : as for nvfp4_harmonize_group.
+ * Errors: as nvfp4_harmonize_group; codes must be 8-byte aligned.
+ */
+nvfp4_status nvfp4_harmonize_requant(uint8_t *codes, uint8_t *sf, int64_t rows_total, int64_t K, int n_modules,
+                                     const int64_t *row_offsets, const float *gscales, float *shared_gscale_out,
+                                     nvfp4_stream_t stream);
+
+/*
+ * Quantize fused into the RMSNorm that produces a layer's input (the norms
+ * stay in BF16 and the GDN layer feeds the normalized residual stream to its
+ * projections: ta-paperlens page, "前提2"), so the normalized activation is
+ * never written out:
+ *   inv_r = the fp32 nearest to 1/sqrt(mean_k x[r,k]^2 + eps)
+ *   y     = bf16(fl32(fl32(x * inv_r) * gamma)),
+ *           gamma = w, or fl32(1 + w) when zero_centered != 0
+ *   codes, sf = nvfp4_quantize(y, gscale)            (bit for bit)
+ * The mean square is evaluated to ~2^-48 relative: inv_r is the correctly
+ * rounded value except when the exact value lies that close to the midpoint
+ * of two floats.
+ *   x        : [rows, K] bf16 or fp32 (dt), row stride ld_x (device); the
+ *              residual stream.
+ *   w        : [K] bf16 norm weight (device, 16-byte aligned).
+ *   eps      : finite and > 0.
+ *   gscale   : 1 float (device), the static global scale of y.
+ *   codes    : [rows, K/2] bytes (device).
+ *   sf       : nvfp4_sf_bytes(rows, K) bytes (device); padding rows zeroed.
+ *   inv_out  : NULL or [rows] floats (device): inv_r.
+ * Errors: NVFP4_ERR_SHAPE for eps <= 0 or not finite; NVFP4_ERR_UNSUPPORTED
+ * when two rows of x and the weight do not fit in one CTA's shared memory
+ * (K above 38592 for bf16 x, 23168 for fp32 x).
+ */
+nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                                    const uint16_t *w, int zero_centered, float eps, const float *gscale,
+                                    uint8_t *codes, uint8_t *sf, float *inv_out, nvfp4_stream_t stream);
+
+/*
  * Synchronizes the device, then reports and clears the library's device error
  * word: *flags receives the OR of the flags kernels recorded since the last
  * call (bit 0: a producer wait ran out, bit 1: an MMA wait ran out, bit 2: an

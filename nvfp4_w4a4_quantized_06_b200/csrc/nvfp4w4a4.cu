@@ -83,9 +83,13 @@ cudaError_t set_cluster_attrs() {
   return e;
 }
 
+constexpr int kSmemOptin = 232448;   // 227 KB, the per-CTA opt-in limit of sm_100
+
 template <typename T>
 cudaError_t set_quant_attrs() {
-  return set_smem(quantize_tma_kernel<T>, QTmaCfg<T>::SMEM_BYTES);
+  cudaError_t e = set_smem(quantize_tma_kernel<T>, QTmaCfg<T>::SMEM_BYTES);
+  if (e == cudaSuccess) e = set_smem(rmsnorm_quantize_kernel<T>, kSmemOptin);
+  return e;
 }
 
 // How many clusters of `size` CTAs of the split-K GEMM fit on the device at once.
@@ -930,6 +934,76 @@ nvfp4_status nvfp4_fp8_quantize(const void *x, nvfp4_in_dtype dt, int64_t n, con
   const cudaError_t e = dt == NVFP4_IN_BF16
                             ? launch_ex(fp8_quantize_kernel<__nv_bfloat16>, (unsigned)blocks, 256u, 0, s, 0, false, p)
                             : launch_ex(fp8_quantize_kernel<float>, (unsigned)blocks, 256u, 0, s, 0, false, p);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  return launched();
+}
+
+nvfp4_status nvfp4_harmonize_requant(uint8_t *codes, uint8_t *sf, int64_t rows_total, int64_t K, int n_modules,
+                                     const int64_t *row_offsets, const float *gscales, float *shared_gscale_out,
+                                     nvfp4_stream_t stream) {
+  if (!codes || !sf || !row_offsets || !gscales || !shared_gscale_out) return NVFP4_ERR_NULL;
+  if (n_modules < 1 || n_modules > kMaxModules || rows_total <= 0 || K <= 0 || K % 64 != 0)
+    return NVFP4_ERR_SHAPE;
+  if (row_offsets[0] != 0 || row_offsets[n_modules] != rows_total) return NVFP4_ERR_SHAPE;
+  for (int m = 0; m < n_modules; ++m)
+    if (row_offsets[m + 1] <= row_offsets[m]) return NVFP4_ERR_SHAPE;
+  if (!aligned16(sf) || (reinterpret_cast<uintptr_t>(codes) & 7)) return NVFP4_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  HarmonizeParams p{};
+  p.sf = sf;
+  p.rows_total = rows_total;
+  p.K = K;
+  p.n = n_modules;
+  for (int m = 0; m <= n_modules; ++m) p.offs[m] = row_offsets[m];
+  p.gs = gscales;
+  p.gstar_out = shared_gscale_out;
+  const int64_t total = rows_total * (K / 16);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
+  harmonize_requant_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p, codes);
+  return launched();
+}
+
+nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                                    const uint16_t *w, int zero_centered, float eps, const float *gscale,
+                                    uint8_t *codes, uint8_t *sf, float *inv_out, nvfp4_stream_t stream) {
+  if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
+  if (rows < 0 || K <= 0 || K % 64 != 0 || ld_x < K || !(eps > 0.0f) || !(eps <= 3.4028235e38f))
+    return NVFP4_ERR_SHAPE;
+  if (!sf || !gscale || !w || (rows > 0 && (!x || !codes))) return NVFP4_ERR_NULL;
+  const int esz = dt == NVFP4_IN_BF16 ? 2 : 4;
+  if ((rows > 0 && (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 7))) || (ld_x * esz) % 16 != 0 ||
+      !aligned16(sf) || !aligned16(w) || (inv_out && (reinterpret_cast<uintptr_t>(inv_out) & 3)))
+    return NVFP4_ERR_ALIGN;
+  int stages = 4;
+  while (stages > 2 && rms_smem_bytes(K, esz, stages) > 56 * 1024) --stages;
+  const int64_t smem = rms_smem_bytes(K, esz, stages);
+  if (smem > kSmemOptin) return NVFP4_ERR_UNSUPPORTED;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  const int64_t pad_rows = pad128(rows) - rows;
+  if (rows == 0 && pad_rows == 0) return NVFP4_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  RmsQuantParams p{x, rows, K, ld_x, reinterpret_cast<const __nv_bfloat16 *>(w), zero_centered ? 1 : 0, eps,
+                   gscale, codes, sf, inv_out, pad_rows, stages, dev->err};
+  int per_sm = 0;
+  cudaError_t e = dt == NVFP4_IN_BF16
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quantize_kernel<__nv_bfloat16>,
+                                                                      kRmsThreads, (size_t)smem)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quantize_kernel<float>,
+                                                                      kRmsThreads, (size_t)smem);
+  if (e != cudaSuccess || per_sm < 1) return NVFP4_ERR_CUDA;
+  int64_t grid = (int64_t)per_sm * dev->sms;
+  if (grid > rows) grid = rows;
+  if (grid < 1) grid = 1;
+  e = dt == NVFP4_IN_BF16
+          ? launch_ex(rmsnorm_quantize_kernel<__nv_bfloat16>, (unsigned)grid, (unsigned)kRmsThreads, (size_t)smem, s, 0,
+                      false, p)
+          : launch_ex(rmsnorm_quantize_kernel<float>, (unsigned)grid, (unsigned)kRmsThreads, (size_t)smem, s, 0, false,
+                      p);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   return launched();
 }

@@ -125,9 +125,9 @@ struct EncodeConsts {
   bool fast;                // g well inside the normal range: products neither overflow nor underflow
 };
 
-__device__ __forceinline__ EncodeConsts encode_consts(const float *gscale) {
+__device__ __forceinline__ EncodeConsts encode_consts_of(float g) {
   EncodeConsts k;
-  k.g = __ldg(gscale);
+  k.g = g;
   k.g6 = __fmul_rn(6.0f, k.g);
   k.rg = __frcp_rn(k.g);
   const float rg6 = __frcp_rn(k.g6);
@@ -136,6 +136,8 @@ __device__ __forceinline__ EncodeConsts encode_consts(const float *gscale) {
   k.fast = k.g >= 8.67361738e-19f && k.g <= 1.15292150e18f;   // 2^-60 .. 2^60
   return k;
 }
+
+__device__ __forceinline__ EncodeConsts encode_consts(const float *gscale) { return encode_consts_of(__ldg(gscale)); }
 
 // Shared table of fl32(1/dec(s)) for every finite non-negative E4M3 byte s;
 // entry 0 is unused (a zero scale short-circuits to zero codes).
@@ -287,6 +289,25 @@ __device__ __forceinline__ void pdl_prologue() {
   if (threadIdx.x == 0) griddep_launch_dependents();
 }
 
+// Zero the scale bytes of `pad_rows` padding rows starting at scale row
+// `first` (fewer than 128 rows of K/16 columns: 32-bit index arithmetic
+// unless K is huge), spread over the whole grid.
+__device__ __forceinline__ void zero_pad_scales(uint8_t *sf, int64_t first, int64_t pad_rows, int64_t K) {
+  const int64_t ncols = K >> 4;
+  const int64_t pad_bytes = pad_rows * ncols;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  if (pad_bytes < (int64_t(1) << 31)) {
+    const uint32_t nc = (uint32_t)ncols;
+    for (uint32_t i = (uint32_t)tid; i < (uint32_t)pad_bytes; i += (uint32_t)nthreads) {
+      const uint32_t rr = i / nc, c = i - rr * nc;
+      sf[sf_index(first + rr, c, K)] = 0;
+    }
+  } else {
+    for (int64_t i = tid; i < pad_bytes; i += nthreads) sf[sf_index(first + i / ncols, i % ncols, K)] = 0;
+  }
+}
+
 // Generic path (any row offset inside a fused buffer, any row count): one
 // warp per 512-column segment of a row, lane l encodes block l of it (32
 // bytes of bf16 per lane, 1 KB contiguous per warp), UNROLL segments loaded
@@ -303,7 +324,6 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   const uint32_t nseg = (uint32_t)((p.K + 511) >> 9);
   const uint32_t units = (uint32_t)p.rows * nseg;
-  const int64_t ncols = p.K >> 4;
   const T *x = static_cast<const T *>(p.x);
   // the encoder constants are read after the first loads are in flight, so
   // the two round trips overlap (few-row calls run a single iteration)
@@ -336,21 +356,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantizeParams p) {
       }
     }
   }
-  // zero the scale bytes of the padding rows this call owns
-  // (fewer than 128 rows of K/16 columns: 32-bit index arithmetic unless K is huge)
-  const int64_t pad_bytes = p.pad_rows * ncols;
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  if (pad_bytes < (int64_t(1) << 31)) {
-    const uint32_t nc = (uint32_t)ncols;
-    for (uint32_t i = (uint32_t)tid; i < (uint32_t)pad_bytes; i += (uint32_t)nthreads) {
-      const uint32_t rr = i / nc, c = i - rr * nc;
-      p.sf[sf_index(p.sf_row0 + p.rows + rr, c, p.K)] = 0;
-    }
-  } else {
-    for (int64_t i = tid; i < pad_bytes; i += nthreads)
-      p.sf[sf_index(p.sf_row0 + p.rows + i / ncols, i % ncols, p.K)] = 0;
-  }
+  zero_pad_scales(p.sf, p.sf_row0 + p.rows, p.pad_rows, p.K);
 }
 
 // Streaming path for calls whose scale rows start on a 128-row boundary and
@@ -746,6 +752,223 @@ __global__ void __launch_bounds__(256) harmonize_kernel(HarmonizeParams p) {
     }
     *w = out;
   }
+}
+
+// Re-quantizing harmonize of a fused group, in place.  Every block of module
+// m is dequantized to fp32 (dec(q) * dec(s) is exact, so fl32(that * g_m) is
+// the exact NVFP4 value rounded once, as the fake-quant kernel writes it) and
+// encoded again against g* = max g_m with the quantize kernels' encoder.
+// Codes and scale bytes both change; padding rows are left as they are.
+// One thread per 16-element block; the decoded values also go to shared
+// memory, where the encoder's rare settling path re-reads them.
+__global__ void __launch_bounds__(256) harmonize_requant_kernel(HarmonizeParams p, uint8_t *codes) {
+  __shared__ float rcp_tab[128];
+  __shared__ float gs[kMaxModules];
+  __shared__ float gstar_s;
+  __shared__ __align__(16) float vals[256][16];
+  fill_rcp_table(rcp_tab);
+  if (threadIdx.x == 0) {
+    float gstar = __ldg(p.gs);
+    for (int m = 0; m < p.n; ++m) {
+      gs[m] = __ldg(p.gs + m);
+      gstar = fmaxf(gstar, gs[m]);
+    }
+    gstar_s = gstar;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.gstar_out = gstar_s;
+  const EncodeConsts kc = encode_consts_of(gstar_s);
+  float *src = vals[threadIdx.x];
+  const int64_t nb = p.K >> 4;
+  const int64_t total = p.rows_total * nb;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / nb, c = i - r * nb;
+    int m = 0;
+    while (m + 1 < p.n && r >= p.offs[m + 1]) ++m;
+    uint8_t *sfp = p.sf + sf_index(r, c, p.K);
+    uint2 *cp = reinterpret_cast<uint2 *>(codes + r * (p.K >> 1) + c * 8);
+    const uint2 cw = *cp;
+    const float ds = e4m3_to_f32(*sfp), g = gs[m];
+    Block16<float> b;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t q = ((e < 8 ? cw.x : cw.y) >> ((e & 7) * 4)) & 0xFu;
+      b.v[e] = __fmul_rn(__fmul_rn(e2m1_to_f32(q), ds), g);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) reinterpret_cast<float4 *>(src)[k] = make_float4(b.v[4 * k], b.v[4 * k + 1], b.v[4 * k + 2], b.v[4 * k + 3]);
+    uint32_t s;
+    *cp = encode16(b, kc, rcp_tab, src, &s);
+    *sfp = static_cast<uint8_t>(s);
+  }
+}
+
+// ------------------------------------------- quantize fused into RMSNorm
+// The BF16 RMSNorm of the residual stream, quantized in the same pass:
+//   inv = the fp32 nearest to 1/sqrt(mean_k x_k^2 + eps)
+//   y_k = bf16(fl32(fl32(x_k * inv) * gamma_k)),  gamma = w or fl32(1 + w)
+// then y quantized like any activation (codes, swizzled scales).  The mean
+// square is accumulated in fp64 (each square exact; relative error of the
+// sum below 2^-46 for rows up to 36K columns), scaled by fl64(1/K), plus
+// eps, and rsqrt (at most one ulp) gives 1/sqrt to ~2^-48: the fp32 rounding
+// then agrees with the exact one except when the exact value lies within
+// that distance of a midpoint between two floats.
+//
+// One CTA of 256 threads per row at a time, persistent over rows
+// blockIdx.x + j * gridDim.x; each row arrives whole in a ring slot by a
+// contiguous bulk copy.  Thread t owns blocks t, t + 256, ... of the row:
+// phase 1 sums their squares (warp shuffles, then one fp64 per warp in
+// shared memory and a CTA barrier), phase 2 writes y back over x in the
+// slot (the encoder's settling path re-reads it) and encodes it.  The slot
+// of row j - 1 is refilled with row j - 1 + STAGES right after the barrier
+// of row j, when every thread is done with it.
+struct RmsQuantParams {
+  const void *x;
+  int64_t rows, K, ld_x;
+  const __nv_bfloat16 *w;   // norm weight [K]
+  int zero_centered;        // gamma = fl32(1 + w) instead of w
+  float eps;
+  const float *gscale;
+  uint8_t *codes;
+  uint8_t *sf;
+  float *inv_out;           // per-row factor [rows], or null
+  int64_t pad_rows;
+  int stages;
+  unsigned *err;
+};
+
+constexpr int kRmsThreads = 256;
+
+// shared memory of the kernel: ring, norm weight, barriers, warp sums, rcp table, abort flag
+__host__ __device__ constexpr int64_t rms_smem_bytes(int64_t K, int esz, int stages) {
+  return stages * K * esz + K * 2 + stages * 8 + 2 * (kRmsThreads / 32) * 8 + 128 * 4 + 16;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRmsThreads, 4) rmsnorm_quantize_kernel(const RmsQuantParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int stages = p.stages;
+  const uint32_t row_bytes = (uint32_t)(p.K * (int64_t)sizeof(T));
+  uint8_t *ring = smem;
+  const uint32_t *wsm = reinterpret_cast<const uint32_t *>(ring + (size_t)stages * row_bytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + (size_t)stages * row_bytes + p.K * 2);
+  double *red = reinterpret_cast<double *>(full + stages);
+  float *rcp_tab = reinterpret_cast<float *>(red + 2 * (kRmsThreads / 32));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(rcp_tab + 128);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const T *x = static_cast<const T *>(p.x);
+  auto issue = [&](int st, int64_t row) {
+    mbar_arrive_expect_tx(&full[st], row_bytes);
+    bulk_load(ring + (size_t)st * row_bytes, x + row * p.ld_x, row_bytes, &full[st]);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  fill_rcp_table(rcp_tab);
+  pdl_prologue();
+  for (int64_t i = tid; i < (p.K >> 3); i += kRmsThreads)
+    reinterpret_cast<uint4 *>(const_cast<uint32_t *>(wsm))[i] = __ldg(reinterpret_cast<const uint4 *>(p.w) + i);
+  __syncthreads();
+  int64_t issued = 0;   // rows of this CTA handed to the copy engine (thread 0's count)
+  if (tid == 0)
+    for (int s = 0; s < stages; ++s) {
+      const int64_t row = blockIdx.x + (int64_t)s * gridDim.x;
+      if (row >= p.rows) break;
+      issue(s, row);
+      ++issued;
+    }
+
+  const EncodeConsts kc = encode_consts(p.gscale);
+  const int nb = (int)(p.K >> 4);
+  const double rk = __drcp_rn((double)p.K);
+  const double eps = (double)p.eps;
+  int st = 0;
+  uint32_t ph = 0;
+  int64_t j = 0;
+  bool stopped = false;
+  for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x, ++j) {
+    const bool ok = mbar_wait(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag);
+    T *sx = reinterpret_cast<T *>(ring + (size_t)st * row_bytes);
+    double acc = 0.0;
+    if (ok) {
+      for (int c = tid; c < nb; c += kRmsThreads) {
+        Block16<T> b;
+        b.load_shared(sx + c * 16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const double v = (double)b.elem(e);
+          acc = fma(v, v, acc);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    double *rw = red + (j & 1) * (kRmsThreads / 32);
+    if (lane == 0) rw[warp] = acc;
+    if (__syncthreads_or(!ok)) {      // a wait ran out: the whole CTA stops here
+      stopped = true;
+      break;
+    }
+    // every thread is done with row j - 1: its slot takes row j - 1 + stages
+    if (tid == 0 && j >= 1) {
+      const int64_t nr = blockIdx.x + (j - 1 + stages) * (int64_t)gridDim.x;
+      if (nr < p.rows) {
+        issue((int)((j - 1) % stages), nr);
+        ++issued;
+      }
+    }
+    double ssq = 0.0;
+#pragma unroll
+    for (int w = 0; w < kRmsThreads / 32; ++w) ssq += rw[w];
+    const float inv = __double2float_rn(rsqrt(fma(ssq, rk, eps)));
+    if (tid == 0 && p.inv_out) p.inv_out[row] = inv;
+
+    uint8_t *crow = p.codes + row * (p.K >> 1);
+    for (int c = tid; c < nb; c += kRmsThreads) {
+      Block16<T> xb;
+      xb.load_shared(sx + c * 16);
+      __nv_bfloat16 *ysrc = reinterpret_cast<__nv_bfloat16 *>(sx + c * 16);
+      const uint4 w0 = reinterpret_cast<const uint4 *>(wsm)[2 * c], w1 = reinterpret_cast<const uint4 *>(wsm)[2 * c + 1];
+      const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      Block16<__nv_bfloat16> yb;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float g0 = __uint_as_float(ww[i] << 16), g1 = __uint_as_float(ww[i] & 0xFFFF0000u);
+        if (p.zero_centered) {
+          g0 = __fadd_rn(1.0f, g0);
+          g1 = __fadd_rn(1.0f, g1);
+        }
+        const float y0 = __fmul_rn(__fmul_rn(xb.elem(2 * i), inv), g0);
+        const float y1 = __fmul_rn(__fmul_rn(xb.elem(2 * i + 1), inv), g1);
+        __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+        yb.w[i] = *reinterpret_cast<uint32_t *>(&h);
+      }
+      reinterpret_cast<uint4 *>(ysrc)[0] = make_uint4(yb.w[0], yb.w[1], yb.w[2], yb.w[3]);
+      reinterpret_cast<uint4 *>(ysrc)[1] = make_uint4(yb.w[4], yb.w[5], yb.w[6], yb.w[7]);
+      uint32_t s;
+      const uint2 word = encode16(yb, kc, rcp_tab, ysrc, &s);
+      *reinterpret_cast<uint2 *>(crow + c * 8) = word;
+      p.sf[sf_index(row, c, p.K)] = static_cast<uint8_t>(s);
+    }
+    fence_proxy_async_shared();       // y was written through the generic proxy; the next copy overwrites it
+    if (++st == stages) {
+      st = 0;
+      ph ^= 1;
+    }
+  }
+  if (stopped) {
+    // let the copies still in flight land before the CTA's memory goes away
+    if (tid == 0) {
+      volatile int never = 0;
+      for (int64_t k = j; k < issued; ++k) mbar_wait(&full[k % stages], (uint32_t)((k / stages) & 1), p.err, ERR_EPILOGUE, &never);
+    }
+    return;
+  }
+  zero_pad_scales(p.sf, p.rows, p.pad_rows, p.K);
 }
 
 }  // namespace nvfp4

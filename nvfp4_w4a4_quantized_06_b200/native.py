@@ -51,13 +51,15 @@ def lib() -> ctypes.CDLL:
         L.w4a4_gdn_gates.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, sz, vp]
         L.nvfp4_fake_quant.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, i64, vp, vp]
         L.nvfp4_fp8_quantize.argtypes = [vp, i32, i64, vp, vp, vp]
+        L.nvfp4_harmonize_requant.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
+        L.nvfp4_rmsnorm_quantize.argtypes = [vp, i32, i64, i64, i64, vp, i32, ctypes.c_float, vp, vp, vp, vp, vp]
         L.nvfp4_selftest_wait_timeout.argtypes = [i64, vp, vp]
         L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
                   "w4a4_gemm", "w4a4_gemm_noalloc", "w4a4_gemm_fused", "w4a4_gdn_gates", "nvfp4_fake_quant", "nvfp4_fp8_quantize",
-                  "nvfp4_selftest_wait_timeout", "nvfp4_last_device_status"):
+                  "nvfp4_harmonize_requant", "nvfp4_rmsnorm_quantize", "nvfp4_selftest_wait_timeout", "nvfp4_last_device_status"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -257,6 +259,40 @@ def fp8_quantize(x: torch.Tensor, scale: torch.Tensor, out: torch.Tensor | None 
     _check("nvfp4_fp8_quantize", lib().nvfp4_fp8_quantize(_ptr(x), _in_dtype(x), x.numel(), _ptr(scale),
                                                           _ptr(out), _stream()))
     return out
+
+
+def harmonize_requant(codes: torch.Tensor, sf: torch.Tensor, K: int, row_offsets, gscales: torch.Tensor,
+                      out: torch.Tensor | None = None) -> torch.Tensor:
+    """Re-quantize a fused group's codes and scales (in place) against one
+    shared global scale; returns g*."""
+    _require_cuda(codes, sf, gscales)
+    offs = (ctypes.c_int64 * len(row_offsets))(*[int(o) for o in row_offsets])
+    out = torch.empty(1, dtype=torch.float32, device=sf.device) if out is None else out
+    _check("nvfp4_harmonize_requant", lib().nvfp4_harmonize_requant(
+        _ptr(codes), _ptr(sf), int(row_offsets[-1]), K, len(row_offsets) - 1, ctypes.cast(offs, ctypes.c_void_p),
+        _ptr(gscales), _ptr(out), _stream()))
+    return out
+
+
+def rmsnorm_quantize(x: torch.Tensor, w: torch.Tensor, eps: float, gscale: torch.Tensor,
+                     zero_centered: bool = False, codes: torch.Tensor | None = None,
+                     sf: torch.Tensor | None = None, inv: torch.Tensor | None = None):
+    """NVFP4 codes and scales of the BF16 RMSNorm of x with weight w (bf16 [K]);
+    returns (codes, sf, inv) where inv [rows] fp32 holds each row's 1/rms."""
+    _require_cuda(x, w, gscale)
+    if w.dtype != torch.bfloat16 or not w.is_contiguous():
+        raise TypeError("the norm weight must be a contiguous bf16 vector")
+    rows, K = x.shape
+    if codes is None:
+        codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(sf_bytes(rows, K), dtype=torch.uint8, device=x.device)
+    if inv is None:
+        inv = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check("nvfp4_rmsnorm_quantize", lib().nvfp4_rmsnorm_quantize(
+        _ptr(x), _in_dtype(x), rows, K, x.stride(0), _ptr(w), 1 if zero_centered else 0, float(eps),
+        _ptr(gscale), _ptr(codes), _ptr(sf), _ptr(inv), _stream()))
+    return codes, sf, inv
 
 
 def selftest_wait_timeout(limit_ns: int = 50_000_000) -> torch.Tensor:

@@ -121,6 +121,16 @@ def make_w(wl: Workload, module: int) -> torch.Tensor:
     return gaussian(wl.modules[module], wl.K, wl.w_seeds[module], wl.w_std, NONE, wl.x_dtype)
 
 
+def norm_weight(K: int, seed: int, zero_centered: bool = False) -> torch.Tensor:
+    """Seeded random-init RMSNorm weight [K] in bf16: 1 + 0.1 N(0,1), or the
+    0.1 N(0,1) offset of the zero-centred form (gamma = 1 + w)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    w = rng.standard_normal(K, dtype=np.float32) * np.float32(0.1)
+    if not zero_centered:
+        w += np.float32(1.0)
+    return torch.from_numpy(w).to(torch.bfloat16)
+
+
 def sample_rows(M: int, n: int, seed: int = 1234) -> np.ndarray:
     """Sorted seeded row sample that always includes the first and last row."""
     if n >= M:

@@ -113,3 +113,29 @@ def test_next_rows_validation(L):
     assert q(FAKE, 0, 16, None, FAKE, None) == 1
     assert q(FAKE + 8, 0, 16, FAKE, FAKE, None) == 3
     assert q(FAKE, 0, 0, None, None, None) == 0                              # empty: nothing to do
+
+
+def test_requant_and_rmsnorm_validation(L):
+    h = L.nvfp4_harmonize_requant
+    offs = (ctypes.c_int64 * 3)(0, 48, 96)
+    bad = (ctypes.c_int64 * 3)(0, 48, 90)
+    po = ctypes.cast(offs, ctypes.c_void_p)
+    assert h(FAKE, FAKE, 96, 256, 2, ctypes.cast(bad, ctypes.c_void_p), FAKE, FAKE, None) == 2
+    assert h(FAKE, FAKE, 96, 100, 2, po, FAKE, FAKE, None) == 2              # K % 64
+    assert h(None, FAKE, 96, 256, 2, po, FAKE, FAKE, None) == 1              # null codes
+    assert h(FAKE + 4, FAKE, 96, 256, 2, po, FAKE, FAKE, None) == 3          # codes not 8-byte aligned
+    r = L.nvfp4_rmsnorm_quantize
+    tail = [FAKE, FAKE, FAKE, None, None]                                     # gscale, codes, sf, inv, stream
+    assert r(FAKE, 0, 4, 256, 256, FAKE, 0, 0.0, *tail) == 2                # eps must be > 0
+    assert r(FAKE, 0, 4, 256, 256, FAKE, 0, float("nan"), *tail) == 2
+    assert r(FAKE, 0, 4, 256, 256, FAKE, 0, float("inf"), *tail) == 2
+    assert r(FAKE, 2, 4, 256, 256, FAKE, 0, 1e-6, *tail) == 4               # dtype
+    assert r(FAKE, 0, 4, 100, 100, FAKE, 0, 1e-6, *tail) == 2               # K % 64
+    assert r(FAKE, 0, 4, 256, 256, None, 0, 1e-6, *tail) == 1               # null weight
+    assert r(FAKE, 0, 4, 256, 256, FAKE + 8, 0, 1e-6, *tail) == 3           # misaligned weight
+    assert r(FAKE, 0, 4, 256, 256, FAKE, 0, 1e-6, FAKE, FAKE, FAKE, FAKE + 2, None) == 3   # misaligned inv
+    # two rows and the weight must fit in one CTA's shared memory
+    assert r(FAKE, 0, 4, 38656, 38656, FAKE, 0, 1e-6, *tail) == 5
+    assert r(FAKE, 1, 4, 23232, 23232, FAKE, 0, 1e-6, *tail) == 5
+    assert r(FAKE, 0, 4, 38592, 38592, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
+    assert r(FAKE, 1, 4, 23168, 23168, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)

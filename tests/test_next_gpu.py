@@ -1,7 +1,7 @@
 """GPU parity of the rows marked "next" against the oracle, through the C ABI:
 the GDN gate projection with its activations fused into the GEMM epilogue,
-fake-quant (Q -> DQ) with its error statistics, and static-scale FP8 E4M3
-quantize."""
+fake-quant (Q -> DQ) with its error statistics, static-scale FP8 E4M3
+quantize, the re-quantizing harmonize and the quantize fused into RMSNorm."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +9,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_06_b200 import native
 from nvfp4_w4a4_quantized_06_b200 import workloads as W
-from parity import f32, to_f32_numpy
+from parity import assert_codes_equal, assert_sf_rows_equal, f32, to_f32_numpy
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -112,3 +112,164 @@ def test_fp8_quantize_bit_exact(in_dtype, scale):
     assert native.last_device_status() == 0
     ref = oracle.fp8_quantize(to_f32_numpy(xt), s)
     assert np.array_equal(q.cpu().numpy(), ref)
+
+
+# ------------------------------------------------- re-quantizing harmonize
+def _quantized_group(mods, K):
+    """Quantize each module with its own scale into one fused buffer, on the
+    GPU and in the oracle; returns both copies."""
+    N = sum(w.shape[0] for w, _ in mods)
+    offs = np.concatenate([[0], np.cumsum([w.shape[0] for w, _ in mods])]).astype(np.int64)
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=DEV)
+    sf = torch.empty(native.sf_bytes(N, K), dtype=torch.uint8, device=DEV)
+    ref_sf = np.zeros(oracle.sf_bytes(N, K), np.uint8)
+    ref_codes = []
+    for m, (w, g) in enumerate(mods):
+        gd = torch.tensor([g], dtype=torch.float32, device=DEV)
+        native.quantize(w.to(DEV), gd, codes=codes[offs[m]:offs[m + 1]], sf=sf, sf_row0=int(offs[m]),
+                        sf_rows_total=N)
+        c, _ = oracle.quantize(to_f32_numpy(w), np.float32(g), sf=ref_sf, sf_row0=int(offs[m]))
+        ref_codes.append(c)
+    torch.cuda.synchronize()
+    assert_codes_equal(codes, np.concatenate(ref_codes))
+    assert np.array_equal(sf.cpu().numpy(), ref_sf)
+    return offs, codes, sf, np.concatenate(ref_codes), ref_sf
+
+
+@pytest.mark.parametrize("case", ["gates_ab", "ragged3", "tiny_ratio"])
+def test_harmonize_requant_matches_oracle(case):
+    if case == "gates_ab":
+        K, specs = 5120, [(48, 1, 0.02), (48, 2, 0.02)]
+    elif case == "ragged3":
+        K, specs = 320, [(33, 3, 0.02), (100, 4, 0.05), (7, 5, 0.004)]
+    else:                                   # one module 2e-5 as large: its scales go subnormal at g*
+        K, specs = 256, [(40, 6, 0.02), (24, 7, 0.02 * 2e-5)]
+    mods = []
+    for rows, seed, std in specs:
+        w = W.gaussian(rows, K, seed=seed, std=std)
+        mods.append((w, oracle.global_scale(to_f32_numpy(w))))
+    offs, codes, sf, rc, rs = _quantized_group(mods, K)
+    gs = torch.tensor([g for _, g in mods], dtype=torch.float32, device=DEV)
+    gstar = native.harmonize_requant(codes, sf, K, offs, gs)
+    ref_codes, ref_sf, ref_gstar = oracle.harmonize_requant(rc, rs, K, offs, [g for _, g in mods])
+    torch.cuda.synchronize()
+    assert f32(gstar) == ref_gstar
+    assert_codes_equal(codes, ref_codes)
+    assert np.array_equal(sf.cpu().numpy(), ref_sf), "scale buffer differs"
+    if case == "tiny_ratio":
+        assert not np.array_equal(ref_codes, rc)        # the case does move codes
+    assert native.last_device_status() == 0
+
+
+def test_harmonize_requant_full_qkv_z_sampled():
+    """The fused qkv+z weight (10240 + 6144 rows, K 5120) re-quantized on the
+    GPU in one launch; a seeded sample of each module's rows checked against
+    the oracle run on just those rows (the operation is row by row)."""
+    wl = W.WORKLOADS["gdn_qkv_z"]
+    K, N = wl.K, wl.N
+    offs = np.concatenate([[0], np.cumsum(wl.modules)]).astype(np.int64)
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=DEV)
+    sf = torch.empty(native.sf_bytes(N, K), dtype=torch.uint8, device=DEV)
+    ws, gs = [], []
+    for m in range(len(wl.modules)):
+        w = W.make_w(wl, m)
+        if m == 1:
+            w = w * 0.37                    # a ratio that is not a power of two
+        ws.append(w)
+        gs.append(oracle.global_scale(to_f32_numpy(w)))
+        native.quantize(w.to(DEV), torch.tensor([gs[m]], device=DEV), codes=codes[offs[m]:offs[m + 1]], sf=sf,
+                        sf_row0=int(offs[m]), sf_rows_total=N)
+    gstar = native.harmonize_requant(codes, sf, K, offs, torch.tensor(gs, device=DEV))
+    samp = [W.sample_rows(wl.modules[m], 96, seed=m) for m in range(len(wl.modules))]
+    sub_offs = np.concatenate([[0], np.cumsum([len(x) for x in samp])])
+    sub_sf = np.zeros(oracle.sf_bytes(int(sub_offs[-1]), K), np.uint8)
+    sub_codes = np.concatenate([oracle.quantize(to_f32_numpy(ws[m][torch.from_numpy(s)]), gs[m], sf=sub_sf,
+                                                sf_row0=int(sub_offs[m]))[0] for m, s in enumerate(samp)])
+    ref_codes, ref_sf, ref_gstar = oracle.harmonize_requant(sub_codes, sub_sf, K, sub_offs, gs)
+    torch.cuda.synchronize()
+    assert f32(gstar) == ref_gstar
+    fused_rows = np.concatenate([offs[m] + s for m, s in enumerate(samp)])
+    assert_codes_equal(codes[torch.from_numpy(fused_rows).to(DEV)], ref_codes)
+    assert_sf_rows_equal(sf, ref_sf, fused_rows, np.arange(len(fused_rows)), K)
+    assert native.last_device_status() == 0
+
+
+# ------------------------------------------ quantize fused into RMSNorm
+def _static_scale(x: torch.Tensor, w: torch.Tensor, eps: float, zero_centered: bool) -> np.float32:
+    """A calibrated static scale for the normalized activation, from torch's
+    own CPU RMSNorm (input preparation only)."""
+    gamma = (1 + w.float()) if zero_centered else w.float()
+    y = torch.nn.functional.rms_norm(x.float(), (x.shape[1],), weight=gamma, eps=eps)
+    return np.float32(y.abs().max().item()) / np.float32(2688.0)
+
+
+def _check_rmsnorm(x_cpu, w_cpu, eps, zero_centered, rows=None):
+    """GPU rmsnorm_quantize of all of x against the oracle on `rows` (all by
+    default): per-row factor bit-exact, codes and scales byte for byte."""
+    g = _static_scale(x_cpu, w_cpu, eps, zero_centered)
+    codes, sf, inv = native.rmsnorm_quantize(x_cpu.to(DEV), w_cpu.to(DEV), eps,
+                                             torch.tensor([g], device=DEV), zero_centered)
+    R, K = x_cpu.shape
+    sel = np.arange(R) if rows is None else rows
+    xs = to_f32_numpy(x_cpu[torch.from_numpy(sel)])
+    wn = to_f32_numpy(w_cpu)
+    rc, rs, _, rinv, near = oracle.rmsnorm_quantize(xs, wn, eps, g, zero_centered)
+    torch.cuda.synchronize()
+    ginv = inv.cpu().numpy()[sel]
+    if near.any():
+        # the exact factor sits within ~2^-45 of a rounding midpoint: either
+        # neighbour is acceptable, and the codes must follow the one chosen
+        idx = np.flatnonzero(near)
+        assert np.all(np.abs(ginv[idx].view(np.int32) - rinv[idx].view(np.int32)) <= 1)
+        rc, rs, _, rinv, _ = oracle.rmsnorm_quantize(xs, wn, eps, g, zero_centered, inv=ginv)
+    assert np.array_equal(ginv.view(np.uint32), rinv.view(np.uint32)), "per-row factor differs"
+    if rows is None:
+        assert_codes_equal(codes, rc)
+        assert np.array_equal(sf.cpu().numpy(), rs), "swizzled scale buffer differs"
+    else:
+        assert_codes_equal(codes[torch.from_numpy(sel).to(DEV)], rc)
+        assert_sf_rows_equal(sf, rs, sel, np.arange(len(sel)), K)
+        if R % 128:
+            pad = oracle.sf_gather(sf.cpu().numpy(), np.arange(R, (R + 127) // 128 * 128), K)
+            assert np.all(pad == 0)
+    assert native.last_device_status() == 0
+
+
+@pytest.mark.parametrize("rows,K,dtype,zc", [
+    (1, 64, torch.bfloat16, False),
+    (33, 320, torch.bfloat16, True),
+    (300, 5120, torch.bfloat16, False),
+    (129, 2048, torch.float32, False),
+    (4096, 5120, torch.bfloat16, True),       # several rows per CTA: the ring refills
+    (2000, 1024, torch.float32, True),
+    (64, 17408, torch.bfloat16, False),       # two stages
+])
+def test_rmsnorm_quantize_matches_oracle(rows, K, dtype, zc):
+    x = W.gaussian(rows, K, seed=rows + K, outliers=W.Outliers("scale", 0.01, 30.0), dtype=dtype)
+    w = W.norm_weight(K, seed=K, zero_centered=zc)
+    _check_rmsnorm(x, w, 1e-6, zc, rows=None if rows * K <= 2_000_000 else W.sample_rows(rows, 256))
+
+
+def test_rmsnorm_quantize_degenerate_rows():
+    """All-zero rows (inv = 1/sqrt(eps)), constant rows, a lone spike, and
+    tiny values next to large ones in one row."""
+    K = 256
+    x = torch.zeros((6, K), dtype=torch.float32)
+    x[1] = 1.875
+    x[2, 17] = 8.0
+    x[3] = torch.linspace(-3, 3, K)
+    x[4, ::2] = 1e-20
+    x[4, 1] = 300.0
+    x[5] = -2.0
+    w = W.norm_weight(K, seed=3)
+    _check_rmsnorm(x.to(torch.bfloat16), w, 0.484375, False)
+    _check_rmsnorm(x, w, 1e-6, True)
+
+
+def test_rmsnorm_quantize_full_prefill_sampled():
+    """The prefill residual (32768 x 5120 bf16) in one launch; 192 seeded rows
+    checked against the oracle, padding rows zero."""
+    wl = W.WORKLOADS["prefill_mlp_gate_up"]
+    x = W.make_x(wl)
+    w = W.norm_weight(wl.K, seed=11)
+    _check_rmsnorm(x, w, 1e-6, False, rows=W.sample_rows(wl.M, 192))
