@@ -421,11 +421,17 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   fill_rcp_table(rcp_tab);
   pdl_prologue();
   __syncthreads();
+  // loader only: stages with a copy issued (bit s) and the parity of the
+  // phase that copy completes (bit s), for draining after a timeout
+  uint32_t pend = 0u, par = 0u;
   if (loader) {
     // the first round of the ring (x is readable: the prologue has waited)
     for (int s = 0; s < C::STAGES; ++s) {
       const uint32_t u = blockIdx.x + (uint32_t)s * gridDim.x;
-      if (u < units) issue(s, u);
+      if (u < units) {
+        issue(s, u);
+        pend |= 1u << s;
+      }
     }
   }
 
@@ -475,12 +481,24 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
       // has released it
       const uint32_t un = u + (uint32_t)C::STAGES * gridDim.x;
       if (un < units) {
-        if (mbar_wait(&empty[st], ph, p.err, ERR_PRODUCER, abort_flag)) issue(st, un);
-        else stop = true;
+        if (mbar_wait(&empty[st], ph, p.err, ERR_PRODUCER, abort_flag)) {
+          issue(st, un);
+          pend |= 1u << st;
+          par = (par & ~(1u << st)) | ((ph ^ 1u) << st);
+        } else {
+          stop = true;
+        }
       }
     }
     if (__any_sync(0xFFFFFFFFu, stop)) break;       // the whole warp leaves together
     if (++st == C::STAGES) { st = 0; ph ^= 1; }
+  }
+  if (loader && *abort_flag) {
+    // a wait ran out: let the copies still in flight land before the CTA's
+    // shared memory goes away (a consumed copy's phase has completed already)
+    volatile int never = 0;
+    for (int s = 0; s < C::STAGES; ++s)
+      if ((pend >> s) & 1u) mbar_wait(&full[s], (par >> s) & 1u, p.err, ERR_PRODUCER, &never);
   }
 }
 
