@@ -513,6 +513,46 @@ def time_oracle(wl, seconds: float = 10.0, rows: int = 128, cols: int = 2048):
                       f"OpenMP threads {oracle.num_threads()}, numpy BLAS threads as configured"}
 
 
+def oracle_table():
+    """The oracle, as it stands, on every configuration on the host cores:
+    the global scale and quantize of each full activation tensor, and the
+    whole linear (activation quantize, float64 dequantize and GEMM) in full
+    for the configurations with at most 4096 activation rows x 128 weight
+    rows of work per K, else on 256 seeded activation rows, extrapolated
+    linearly in M.  Weight preparation is untimed.  No GPU is used."""
+    import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    table = []
+    for name, wl in W.WORKLOADS.items():
+        x = W.make_x(wl).float().numpy()
+        t0 = time.perf_counter()
+        gx = oracle.global_scale(x)
+        oracle.quantize(x, gx)
+        tq = time.perf_counter() - t0
+        K, N = wl.K, wl.N
+        offs = np.concatenate([[0], np.cumsum(wl.modules)]).astype(np.int64)
+        wsf = np.zeros(oracle.sf_bytes(N, K), np.uint8)
+        wcs, gws = [], []
+        for m in range(len(wl.modules)):
+            w = W.make_w(wl, m).float().numpy()
+            g = oracle.global_scale(w)
+            wcs.append(oracle.quantize(w, g, sf=wsf, sf_row0=int(offs[m]))[0])
+            gws.append(g)
+        gw = oracle.harmonize(wsf, K, offs, gws) if len(gws) > 1 else gws[0]
+        wc = np.concatenate(wcs)
+        full = wl.M * N <= 4096 * 128
+        rows = np.arange(wl.M) if full else W.sample_rows(wl.M, 256)
+        t0 = time.perf_counter()
+        oracle.linear_reference(x[rows], gx, wc, wsf, gw)
+        tg = (time.perf_counter() - t0) * (wl.M / len(rows))
+        table.append({"workload": f"{name} {wl.M}x{N}x{K}", "quantize_s": round(tq, 3),
+                      "quantize_gbs": round(wl.M * K * (2.0 if wl.x_dtype == torch.bfloat16 else 4.0) / tq / 1e9, 3),
+                      "linear_s": round(tg, 3), "linear_gflops": round(wl.flops / tg / 1e9, 2),
+                      "linear_rows": "all" if full else f"{len(rows)} of {wl.M}, extrapolated"})
+        del x, wcs, wc, wsf
+    return {"oracle_table": table, "cores": cores, "openmp_threads": oracle.num_threads()}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -551,8 +591,14 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="time the CPU oracle on every configuration (host cores only) and exit")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+
+    if args.oracle_table:
+        print(json.dumps(oracle_table()), flush=True)
+        return
 
     if args.impl == "reference":
         out = run_reference(args)
