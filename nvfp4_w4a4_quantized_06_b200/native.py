@@ -100,6 +100,45 @@ def _require_cuda(*ts: torch.Tensor) -> None:
             raise ValueError("tensors must live on the GPU")
 
 
+# Layout checks: the C ABI takes bare pointers and sizes, so the binding
+# makes sure every tensor really has the layout and size those imply before
+# any pointer reaches the library (a short buffer would be written past its end).
+def _mat(name: str, t: torch.Tensor, rows: int | None = None, cols: int | None = None) -> None:
+    """A row-major matrix view: 2-D, unit column stride, any row stride."""
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    if (rows is not None and t.shape[0] != rows) or (cols is not None and t.shape[1] != cols):
+        raise ValueError(f"{name} must be [{rows}, {cols}], got {tuple(t.shape)}")
+    if t.numel() and t.stride(1) != 1:
+        raise ValueError(f"{name} must have unit column stride")
+
+
+def _codes(name: str, t: torch.Tensor, rows: int, K: int) -> None:
+    """Packed NVFP4 codes of a [rows, K] tensor: uint8 [rows, K/2], row stride K/2."""
+    if t.dtype != torch.uint8:
+        raise TypeError(f"{name} must be uint8, got {t.dtype}")
+    _mat(name, t, rows, K // 2)
+    if rows > 1 and t.stride(0) != K // 2:
+        raise ValueError(f"{name} must have row stride K/2 = {K // 2}")
+
+
+def _buf(name: str, t: torch.Tensor, dtype: torch.dtype, n: int) -> None:
+    """A contiguous buffer of at least n elements of dtype."""
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {n}")
+
+
+def _offsets(row_offsets) -> list[int]:
+    offs = [int(o) for o in row_offsets]
+    if len(offs) < 2:
+        raise ValueError("row_offsets needs at least two entries")
+    return offs
+
+
 def codes_bytes(rows: int, K: int) -> int:
     return int(lib().nvfp4_codes_bytes(rows, K))
 
@@ -110,7 +149,10 @@ def sf_bytes(rows: int, K: int) -> int:
 
 def amax_gscale(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """Per-tensor global scale amax/(6*448) as a 1-element fp32 device tensor."""
-    _require_cuda(x)
+    _mat("x", x)
+    if out is not None:
+        _buf("out", out, torch.float32, 1)
+    _require_cuda(x, out)
     rows, K = x.shape
     out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
     _check("nvfp4_amax_gscale", lib().nvfp4_amax_gscale(_ptr(x), _in_dtype(x), rows, K, x.stride(0),
@@ -121,9 +163,15 @@ def amax_gscale(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tenso
 def quantize(x: torch.Tensor, gscale: torch.Tensor, codes: torch.Tensor | None = None,
              sf: torch.Tensor | None = None, sf_row0: int = 0, sf_rows_total: int | None = None):
     """NVFP4-quantize x [rows, K]; returns (codes [rows, K/2] uint8, sf uint8 swizzled)."""
-    _require_cuda(x, gscale)
+    _mat("x", x)
     rows, K = x.shape
     total = rows if sf_rows_total is None else sf_rows_total
+    _buf("gscale", gscale, torch.float32, 1)
+    if codes is not None:
+        _codes("codes", codes, rows, K)
+    if sf is not None:
+        _buf("sf", sf, torch.uint8, sf_bytes(total, K))
+    _require_cuda(x, gscale, codes, sf)
     if codes is None:
         codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
     if sf is None:
@@ -136,8 +184,13 @@ def quantize(x: torch.Tensor, gscale: torch.Tensor, codes: torch.Tensor | None =
 def harmonize(sf: torch.Tensor, rows_total: int, K: int, row_offsets, gscales: torch.Tensor,
               out: torch.Tensor | None = None) -> torch.Tensor:
     """Rewrite a fused group's scales to one shared global scale; returns g*."""
-    _require_cuda(sf, gscales)
-    offs = (ctypes.c_int64 * len(row_offsets))(*[int(o) for o in row_offsets])
+    row_offsets = _offsets(row_offsets)
+    _buf("sf", sf, torch.uint8, sf_bytes(rows_total, K))
+    _buf("gscales", gscales, torch.float32, len(row_offsets) - 1)
+    if out is not None:
+        _buf("out", out, torch.float32, 1)
+    _require_cuda(sf, gscales, out)
+    offs = (ctypes.c_int64 * len(row_offsets))(*row_offsets)
     out = torch.empty(1, dtype=torch.float32, device=sf.device) if out is None else out
     _check("nvfp4_harmonize_group", lib().nvfp4_harmonize_group(
         _ptr(sf), rows_total, K, len(row_offsets) - 1, ctypes.cast(offs, ctypes.c_void_p),
@@ -148,9 +201,21 @@ def harmonize(sf: torch.Tensor, rows_total: int, K: int, row_offsets, gscales: t
 def gemm(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, out_dtype=torch.bfloat16,
          out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
     """Y[M, N] = (ga*gb) * dec(A) @ dec(B)^T on pre-quantized NVFP4 operands."""
-    _require_cuda(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale)
+    _mat("a_codes", a_codes)
+    _mat("b_codes", b_codes)
     M, K = a_codes.shape[0], a_codes.shape[1] * 2
     N = b_codes.shape[0]
+    _codes("a_codes", a_codes, M, K)
+    _codes("b_codes", b_codes, N, K)
+    _buf("a_sf", a_sf, torch.uint8, sf_bytes(M, K))
+    _buf("b_sf", b_sf, torch.uint8, sf_bytes(N, K))
+    _buf("a_gscale", a_gscale, torch.float32, 1)
+    _buf("b_gscale", b_gscale, torch.float32, 1)
+    if out is not None:
+        _mat("out", out, M, N)
+    if workspace is not None:
+        _buf("workspace", workspace, torch.uint8, 0)
+    _require_cuda(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, out, workspace)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=a_codes.device)
     need = int(lib().nvfp4_gemm_workspace_bytes(M, N, K))
@@ -163,6 +228,24 @@ def gemm(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, out_dtype=torch.bfloa
     return out
 
 
+def _linear_args(x, x_gscale, w_codes, w_sf, w_gscale, out, workspace=None):
+    """Check the operands of a linear-type call; returns (M, K, N)."""
+    _mat("x", x)
+    M, K = x.shape
+    _mat("w_codes", w_codes)
+    N = w_codes.shape[0]
+    _codes("w_codes", w_codes, N, K)
+    _buf("w_sf", w_sf, torch.uint8, sf_bytes(N, K))
+    _buf("x_gscale", x_gscale, torch.float32, 1)
+    _buf("w_gscale", w_gscale, torch.float32, 1)
+    if out is not None:
+        _mat("out", out, M, N)
+    if workspace is not None:
+        _buf("workspace", workspace, torch.uint8, 0)
+    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale, out, workspace)
+    return M, K, N
+
+
 def linear_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().w4a4_gemm_workspace_bytes(M, N, K))
 
@@ -171,9 +254,7 @@ def linear(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf:
            w_gscale: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
            workspace: torch.Tensor | None = None) -> torch.Tensor:
     """The W4A4 linear: on-the-fly NVFP4 quantize of x, then the block-scaled GEMM."""
-    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
-    M, K = x.shape
-    N = w_codes.shape[0]
+    M, K, N = _linear_args(x, x_gscale, w_codes, w_sf, w_gscale, out, workspace)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
     if workspace is None:
@@ -191,9 +272,7 @@ def linear_noalloc(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tenso
     """The W4A4 linear without a caller workspace: the library's fixed 8 MiB
     scratch buffer holds the quantized activation and split-K partials (for
     callers that cannot allocate device memory at the point of use)."""
-    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
-    M, K = x.shape
-    N = w_codes.shape[0]
+    M, K, N = _linear_args(x, x_gscale, w_codes, w_sf, w_gscale, out)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
     _check("w4a4_gemm_noalloc", lib().w4a4_gemm_noalloc(
@@ -206,9 +285,7 @@ def linear_fused(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor,
                  w_gscale: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
     """The decode-shaped layer (M <= 128) with the activation quantized inside
     the GEMM kernel; bit-identical to linear()."""
-    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
-    M, K = x.shape
-    N = w_codes.shape[0]
+    M, K, N = _linear_args(x, x_gscale, w_codes, w_sf, w_gscale, out)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
     _check("w4a4_gemm_fused", lib().w4a4_gemm_fused(
@@ -222,9 +299,9 @@ def gdn_gates(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_
               workspace: torch.Tensor | None = None) -> torch.Tensor:
     """The fused GDN gate projection: [M, N] float32 with alpha = exp(-softplus(a))
     in columns [0, n_a) and beta = sigmoid(b) in the rest."""
-    _require_cuda(x, x_gscale, w_codes, w_sf, w_gscale)
-    M, K = x.shape
-    N = w_codes.shape[0]
+    if out is not None and out.dtype != torch.float32:
+        raise TypeError(f"out must be float32, got {out.dtype}")
+    M, K, N = _linear_args(x, x_gscale, w_codes, w_sf, w_gscale, out, workspace)
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=x.device)
     if workspace is None:
@@ -238,7 +315,11 @@ def gdn_gates(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_
 def fake_quant(x: torch.Tensor, gscale: torch.Tensor, out_dtype=torch.float32,
                stats: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
     """Quantize-then-dequantize x; returns (values, [sum sq error, sum sq x] float64)."""
-    _require_cuda(x, gscale)
+    _mat("x", x)
+    _buf("gscale", gscale, torch.float32, 1)
+    if stats is not None:
+        _buf("stats", stats, torch.float64, 2)
+    _require_cuda(x, gscale, stats)
     rows, K = x.shape
     out = torch.empty((rows, K), dtype=out_dtype, device=x.device)
     if stats is None:
@@ -251,9 +332,12 @@ def fake_quant(x: torch.Tensor, gscale: torch.Tensor, out_dtype=torch.float32,
 
 def fp8_quantize(x: torch.Tensor, scale: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """FP8 E4M3 codes (uint8, sign in bit 7) of x / scale, x contiguous."""
-    _require_cuda(x, scale)
     if not x.is_contiguous():
         raise ValueError("x must be contiguous")
+    _buf("scale", scale, torch.float32, 1)
+    if out is not None:
+        _buf("out", out, torch.uint8, x.numel())
+    _require_cuda(x, scale, out)
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check("nvfp4_fp8_quantize", lib().nvfp4_fp8_quantize(_ptr(x), _in_dtype(x), x.numel(), _ptr(scale),
@@ -265,8 +349,14 @@ def harmonize_requant(codes: torch.Tensor, sf: torch.Tensor, K: int, row_offsets
                       out: torch.Tensor | None = None) -> torch.Tensor:
     """Re-quantize a fused group's codes and scales (in place) against one
     shared global scale; returns g*."""
-    _require_cuda(codes, sf, gscales)
-    offs = (ctypes.c_int64 * len(row_offsets))(*[int(o) for o in row_offsets])
+    row_offsets = _offsets(row_offsets)
+    _codes("codes", codes, row_offsets[-1], K)
+    _buf("sf", sf, torch.uint8, sf_bytes(row_offsets[-1], K))
+    _buf("gscales", gscales, torch.float32, len(row_offsets) - 1)
+    if out is not None:
+        _buf("out", out, torch.float32, 1)
+    _require_cuda(codes, sf, gscales, out)
+    offs = (ctypes.c_int64 * len(row_offsets))(*row_offsets)
     out = torch.empty(1, dtype=torch.float32, device=sf.device) if out is None else out
     _check("nvfp4_harmonize_requant", lib().nvfp4_harmonize_requant(
         _ptr(codes), _ptr(sf), int(row_offsets[-1]), K, len(row_offsets) - 1, ctypes.cast(offs, ctypes.c_void_p),
@@ -279,10 +369,18 @@ def rmsnorm_quantize(x: torch.Tensor, w: torch.Tensor, eps: float, gscale: torch
                      sf: torch.Tensor | None = None, inv: torch.Tensor | None = None):
     """NVFP4 codes and scales of the BF16 RMSNorm of x with weight w (bf16 [K]);
     returns (codes, sf, inv) where inv [rows] fp32 holds each row's 1/rms."""
-    _require_cuda(x, w, gscale)
-    if w.dtype != torch.bfloat16 or not w.is_contiguous():
-        raise TypeError("the norm weight must be a contiguous bf16 vector")
+    _mat("x", x)
     rows, K = x.shape
+    if w.dtype != torch.bfloat16 or not w.is_contiguous() or w.numel() != K:
+        raise TypeError(f"the norm weight must be a contiguous bf16 vector of {K} elements")
+    _buf("gscale", gscale, torch.float32, 1)
+    if codes is not None:
+        _codes("codes", codes, rows, K)
+    if sf is not None:
+        _buf("sf", sf, torch.uint8, sf_bytes(rows, K))
+    if inv is not None:
+        _buf("inv", inv, torch.float32, rows)
+    _require_cuda(x, w, gscale, codes, sf, inv)
     if codes is None:
         codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
     if sf is None:
