@@ -2,8 +2,9 @@
 // activation/weight quantize (E2M1 codes + swizzled E4M3 block scales; a
 // TMA-fed streaming kernel and a generic per-row kernel), fused-group
 // global-scale harmonization, and the rows built on the same encoder:
-// fake-quant (quantize then dequantize, with error sums) and static-scale
-// FP8 E4M3 quantize.
+// fake-quant (quantize then dequantize, with error sums), static-scale FP8
+// E4M3 quantize, the re-quantizing harmonize, and the quantize fused into
+// the RMSNorm that produces an activation.
 //
 // Format (web pages on arXiv 2609.04098; ta-paperlens page, section "前提1";
 // arxiv-wiki page, "접근 방법"): 4-bit E2M1 values, one E4M3 scale per 16
