@@ -122,3 +122,24 @@ def test_scale_encoder_equals_the_division_for_every_bf16_amax():
         assert np.array_equal(got, want), g
         settled += int(diff.sum())
     assert settled > 0
+
+
+def test_fp8_encoder_equals_the_division_for_every_bf16_value():
+    """The FP8 KV quantize uses the same scheme: E4M3 of x * fl32(1/s) widened
+    both ways, settled against the midpoint of the two candidates."""
+    settled = 0
+    for s in GLOBAL_SCALES:
+        rs = F32(1) / s
+        with np.errstate(over="ignore"):
+            lo = e4m3_code(X_ALL * (rs * WIDEN_LO))
+            hi = e4m3_code(X_ALL * (rs * WIDEN_HI))
+            want = e4m3_code(X_ALL / s)
+        assert np.all(lo <= want) and np.all(want <= hi) and np.all(hi - lo <= 1), s
+        diff = lo != hi
+        mid = ((E4M3_VALUES[lo].astype(np.float32) + E4M3_VALUES[np.minimum(hi, 126)].astype(np.float32))
+               * F32(0.5)).astype(np.float32)
+        got = lo.copy()
+        got[diff] = pick(lo[diff], hi[diff], settle(X_ALL[diff], np.full(int(diff.sum()), s, np.float32), mid[diff]))
+        assert np.array_equal(got, want), s
+        settled += int(diff.sum())
+    assert settled > 0
