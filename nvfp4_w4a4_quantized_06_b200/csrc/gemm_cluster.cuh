@@ -53,7 +53,7 @@ __device__ __forceinline__ float gate_write(float b) { return 1.0f / (1.0f + exp
 // FUSED: the activation (the B operand of decode-shaped products) is read
 // as bf16/fp32 and quantized inside the kernel by QWARPS extra warps, which
 // write the codes straight into the MMA's swizzled B tiles and the scale
-// bytes into the B scale atoms ("quantize in the producer").
+// bytes into the B scale atoms (the quantize fused into the GEMM's producer).
 template <int BN, bool FUSED = false>
 struct ClusterCfg {
   static constexpr int BM = 128;
