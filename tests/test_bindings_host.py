@@ -122,3 +122,23 @@ def test_group_and_next_row_layouts():
         native.amax_gscale(x)
     with pytest.raises(TypeError, match="float32"):
         native.amax_gscale(x, out=torch.zeros(1, dtype=torch.float64))
+
+
+def test_every_entry_point_has_a_ctypes_signature():
+    """Every function the header declares has its argument and result types
+    set in the binding (an unset signature would pass 64-bit sizes and
+    pointers as C ints)."""
+    import ctypes
+    import os
+    import re
+    header = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "nvfp4w4a4.h")
+    text = re.sub(r"/\*.*?\*/", "", open(header).read(), flags=re.S)
+    names = sorted(set(re.findall(r"^[A-Za-z_][A-Za-z0-9_ \*]*?\b((?:nvfp4|w4a4)_[a-z0-9_]+)\s*\(", text, re.M)))
+    L = native.lib()
+    assert len(names) >= 18
+    missing = [n for n in names if getattr(L, n).argtypes is None]
+    assert not missing, missing
+    # the functions that return something other than a status code say so
+    wide = [n for n in names if n.endswith("_bytes") or n in ("nvfp4_launch_count", "nvfp4_status_string")]
+    untyped = [n for n in wide if getattr(L, n).restype is ctypes.c_int]
+    assert wide and not untyped, untyped
