@@ -65,9 +65,20 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+# NVFP4_DEBUG=1: after every call, synchronize and read the device error word,
+# so that a kernel whose bounded wait ran out is reported by the call that
+# launched it (off by default: it serializes the host with the GPU, and it
+# cannot be used while a CUDA graph is being captured).
+DEBUG = os.environ.get("NVFP4_DEBUG", "0") not in ("", "0")
+
+
 def _check(fn: str, status: int) -> None:
     if status != 0:
         raise Nvfp4Error(fn, status)
+    if DEBUG:
+        flags = last_device_status()
+        if flags:
+            raise Nvfp4Error(f"{fn} (device error flags {flags:#x})", 6)
 
 
 def _stream() -> int:

@@ -142,3 +142,19 @@ def test_every_entry_point_has_a_ctypes_signature():
     wide = [n for n in names if n.endswith("_bytes") or n in ("nvfp4_launch_count", "nvfp4_status_string")]
     untyped = [n for n in wide if getattr(L, n).restype is ctypes.c_int]
     assert wide and not untyped, untyped
+
+
+def test_debug_mode_reports_device_flags_at_the_call(monkeypatch):
+    """With NVFP4_DEBUG set, a call that left a device error flag raises at
+    once, naming the entry point; without it, flags wait for the next
+    explicit status read."""
+    monkeypatch.setattr(native, "last_device_status", lambda: 4)
+    monkeypatch.setattr(native, "DEBUG", False)
+    native._check("nvfp4_quantize", 0)
+    monkeypatch.setattr(native, "DEBUG", True)
+    with pytest.raises(native.Nvfp4Error, match=r"nvfp4_quantize \(device error flags 0x4\)"):
+        native._check("nvfp4_quantize", 0)
+    with pytest.raises(native.Nvfp4Error, match="bad shape"):
+        native._check("nvfp4_quantize", 2)
+    monkeypatch.setattr(native, "last_device_status", lambda: 0)
+    native._check("nvfp4_quantize", 0)
