@@ -349,6 +349,22 @@ nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t ro
                                     uint8_t *codes, uint8_t *sf, float *inv_out, nvfp4_stream_t stream);
 
 /*
+ * Diagnostic: the launch plan the GEMM entry points choose for an M x N x K
+ * product on a device with `sms` SMs, `pair_clusters` co-resident CTA pairs of
+ * the pair GEMM and split_clusters[bn][c] co-resident split-K clusters of c
+ * CTAs (bn index 0, 1, 2 for an MMA N of 32, 64, 128; c = 0..8; NULL = no
+ * cluster support).  The entry points take these numbers from the CUDA
+ * occupancy calculator once per device; this call takes them as arguments
+ * and touches no device, so the planning can be checked anywhere.
+ *   out[8] (host): kind (0 single-CTA kernel, 1 CTA pairs, 2 split-K over a
+ *          cluster), MMA N, swap (1: the activation is the MMA's N operand),
+ *          K splits, grid CTAs, tiles of the 128/256-row operand, tiles of the
+ *          other operand, K stages of 256 elements.
+ */
+nvfp4_status nvfp4_plan_for(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters,
+                            const int *split_clusters, int *out);
+
+/*
  * Synchronizes the device, then reports and clears the library's device error
  * word: *flags receives the OR of the flags kernels recorded since the last
  * call (bit 0: a producer wait ran out, bit 1: an MMA wait ran out, bit 2: an

@@ -1008,6 +1008,28 @@ nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t ro
   return launched();
 }
 
+nvfp4_status nvfp4_plan_for(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters, const int *split_clusters,
+                            int *out) {
+  if (!out) return NVFP4_ERR_NULL;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0 || sms <= 0 || pair_clusters < 0) return NVFP4_ERR_SHAPE;
+  DeviceState d{};
+  d.sms = sms;
+  d.pair_clusters = pair_clusters;
+  if (split_clusters)
+    for (int b = 0; b < 3; ++b)
+      for (int c = 0; c <= kMaxSplitCluster; ++c) d.split_clusters[b][c] = split_clusters[b * (kMaxSplitCluster + 1) + c];
+  const Plan pl = make_plan(M, N, K, d);
+  out[0] = (int)pl.kind;
+  out[1] = pl.bn;
+  out[2] = pl.swap ? 1 : 0;
+  out[3] = pl.splits;
+  out[4] = pl.grid;
+  out[5] = pl.tiles_a;
+  out[6] = pl.tiles_b;
+  out[7] = pl.kstages;
+  return NVFP4_OK;
+}
+
 nvfp4_status nvfp4_selftest_wait_timeout(int64_t limit_ns, int *result_dev, nvfp4_stream_t stream) {
   if (!result_dev) return NVFP4_ERR_NULL;
   if (limit_ns <= 0 || limit_ns > 2000000000LL) return NVFP4_ERR_SHAPE;

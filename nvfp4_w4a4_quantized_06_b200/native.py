@@ -54,12 +54,13 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_harmonize_requant.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
         L.nvfp4_rmsnorm_quantize.argtypes = [vp, i32, i64, i64, i64, vp, i32, ctypes.c_float, vp, vp, vp, vp, vp]
         L.nvfp4_selftest_wait_timeout.argtypes = [i64, vp, vp]
+        L.nvfp4_plan_for.argtypes = [i64, i64, i64, i32, i32, vp, vp]
         L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
                   "w4a4_gemm", "w4a4_gemm_noalloc", "w4a4_gemm_fused", "w4a4_gdn_gates", "nvfp4_fake_quant", "nvfp4_fp8_quantize",
-                  "nvfp4_harmonize_requant", "nvfp4_rmsnorm_quantize", "nvfp4_selftest_wait_timeout", "nvfp4_last_device_status"):
+                  "nvfp4_harmonize_requant", "nvfp4_rmsnorm_quantize", "nvfp4_selftest_wait_timeout", "nvfp4_plan_for", "nvfp4_last_device_status"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -402,6 +403,30 @@ def rmsnorm_quantize(x: torch.Tensor, w: torch.Tensor, eps: float, gscale: torch
         _ptr(x), _in_dtype(x), rows, K, x.stride(0), _ptr(w), 1 if zero_centered else 0, float(eps),
         _ptr(gscale), _ptr(codes), _ptr(sf), _ptr(inv), _stream()))
     return codes, sf, inv
+
+
+PLAN_KINDS = {0: "single", 1: "pair", 2: "cluster"}
+
+
+def plan_for(M: int, N: int, K: int, sms: int = 148, pair_clusters: int = 0, split_clusters=None) -> dict:
+    """The GEMM launch plan for an M x N x K product given the device's
+    occupancy figures (no device is touched); split_clusters[bn][c] for MMA N
+    32/64/128 and cluster sizes c = 0..8."""
+    table = None
+    if split_clusters is not None:
+        flat = [int(v) for row in split_clusters for v in row]
+        if len(flat) != 27:
+            raise ValueError("split_clusters must be 3 rows of 9 counts")
+        table = (ctypes.c_int * 27)(*flat)
+    out = (ctypes.c_int * 8)()
+    _check("nvfp4_plan_for", lib().nvfp4_plan_for(M, N, K, sms, pair_clusters,
+                                                  None if table is None else ctypes.cast(table, ctypes.c_void_p),
+                                                  ctypes.cast(out, ctypes.c_void_p)))
+    keys = ("kind", "bn", "swap", "splits", "grid", "tiles_a", "tiles_b", "kstages")
+    d = dict(zip(keys, list(out)))
+    d["kind"] = PLAN_KINDS[d["kind"]]
+    d["swap"] = bool(d["swap"])
+    return d
 
 
 def selftest_wait_timeout(limit_ns: int = 50_000_000) -> torch.Tensor:
