@@ -1,5 +1,7 @@
 import os
+import shutil
 import sys
+import tempfile
 
 import pytest
 
@@ -18,3 +20,14 @@ def oracle():
     import oracle as _oracle
     _oracle.build()
     return _oracle
+
+
+@pytest.fixture
+def work_dir():
+    """A scratch directory inside the repository's ignored _build/ folder,
+    removed after the test."""
+    base = os.path.join(ROOT, "_build", "tests")
+    os.makedirs(base, exist_ok=True)
+    d = tempfile.mkdtemp(dir=base)
+    yield d
+    shutil.rmtree(d, ignore_errors=True)

@@ -1,6 +1,8 @@
 """Save/load of the shipped artefacts (no GPU needed): NVFP4 weights from the
 CPU oracle's quantize, a harmonized fused group, and static FP8 KV scales
 round-trip byte for byte; damaged files are refused with a clear error."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -31,10 +33,10 @@ def _group(K=256):
                               torch.tensor([gstar], dtype=torch.float32), (48, 48))
 
 
-def test_round_trip(tmp_path):
+def test_round_trip(work_dir):
     layers = {"mlp.gate_up": _layer(130, 320, 1), "gdn.in_proj_ba": _group()}
     kv = {"layer3.k": 0.0125, "layer3.v": 0.031}
-    p = str(tmp_path / "model.nvfp4")
+    p = os.path.join(work_dir, "model.nvfp4")
     ck.save(p, layers, kv)
     got, kv2 = ck.load(p)
     assert set(got) == set(layers) and kv2 == pytest.approx(kv, rel=0, abs=1e-9)
@@ -44,9 +46,9 @@ def test_round_trip(tmp_path):
         assert r.module_rows == q.module_rows and (r.N, r.K) == (q.N, q.K)
 
 
-def test_damaged_files_are_refused(tmp_path):
+def test_damaged_files_are_refused(work_dir):
     q = _layer(64, 256, 3)
-    p = str(tmp_path / "m.nvfp4")
+    p = os.path.join(work_dir, "m.nvfp4")
     with pytest.raises(ValueError, match="scales"):
         ck.save(p, {"a": ck.QuantizedLinear(q.codes, q.sf[:-1], q.gscale)})
     with pytest.raises(ValueError, match="multiple of 64"):
