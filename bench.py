@@ -60,15 +60,18 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
+        self.path = os.path.join(ROOT, "_build", f"nvfp4_clocks_{os.getpid()}.csv")
 
     def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
+            if os.path.exists(self.path):
+                os.unlink(self.path)
 
     def stop(self):
         if self.proc is None:
