@@ -94,9 +94,21 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         loaded = [s for s in sm if s > 0.5 * smax] or sm
+        cap = sum(1 for r in rows if r[8].lower().startswith("active")) / len(rows)
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
-                                                          if r[3].replace(".", "").isdigit())}
+                "samples": len(rows), "power_cap_share": round(cap, 3),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def fp4_peak_for(pk, clocks):
+    """The dense FP4 denominator for a kernel timed in this run: 4 x the
+    measured BF16 GEMM rate (the nominal FP4/BF16 ratio), taken at the burst
+    figure unless the power cap held the clocks for most of the timed region,
+    in which case the sustained (power-capped) figure applies."""
+    share = clocks.get("power_cap_share") or 0.0
+    if "sw_power_cap" in clocks.get("reasons", []) and share > 0.5:
+        return pk["bf16_tflops_sustained"] * FP4_OVER_BF16, "sustained"
+    return pk["bf16_tflops"] * FP4_OVER_BF16, "burst"
 
 
 # ---------------------------------------------------------------- helpers
@@ -135,12 +147,16 @@ def quantized_weight(wl, dev):
     return codes, sf, gw
 
 
-def kernel_src_hash():
-    """Digest of the sources the CTA-pair GEMM is compiled from (its launch
-    shape lives in nvfp4w4a4.cu's plan; a change there that touches the pair
-    path must refresh profiles/dram_traffic.json by hand)."""
+GEMM_SOURCES = ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")
+QUANT_SOURCES = ("quantize.cuh", "ptx.cuh")
+
+
+def kernel_src_hash(files=GEMM_SOURCES):
+    """Digest of the sources a kernel is compiled from (its launch shape lives
+    in nvfp4w4a4.cu's plan; a change there that touches the kernel's launch
+    must refresh profiles/dram_traffic.json by hand)."""
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh"):
+    for f in files:
         text = open(os.path.join(ROOT, "nvfp4_w4a4_quantized_06_b200", "csrc", f), encoding="utf-8").read()
         # comments do not change the kernel: hash the code only
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -150,14 +166,14 @@ def kernel_src_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(name: str):
+def recorded_traffic(name: str, files=GEMM_SOURCES):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path)).get(name)
-    if not d or d.get("src_hash") != kernel_src_hash():
+    if not d or d.get("src_hash") != kernel_src_hash(files):
         return None
     return d.get("bytes_per_launch")
 
@@ -226,15 +242,15 @@ def run_native(args, rank, world, dev):
     value = job_throughput(flops, world, ms_per_step)
     pk = peaks()
     tq_ms, tg_ms = sq / args.steps, sg / args.steps
-    # the GEMM runs back to back for the whole timed region (a second or more
-    # under the power cap), so its denominator is the sustained figure
-    fp4_peak = pk["bf16_tflops_sustained"] * FP4_OVER_BF16
+    fp4_peak, peak_kind = fp4_peak_for(pk, clocks)
     fp4_peak_burst = pk["bf16_tflops"] * FP4_OVER_BF16
+    fp4_peak_sust = pk["bf16_tflops_sustained"] * FP4_OVER_BF16
     gemm_tflops = flops / (tg_ms * 1e-3) / 1e12
     q_gbs = quant_bytes(M, K) / (tq_ms * 1e-3) / 1e9
 
     # ---- end to end through the public one-call API, host buffers
-    e2e = None if args.no_e2e else measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world)
+    e2e = None if args.no_e2e else measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world,
+                                               steps=min(args.steps, 50))
 
     also = {}
     if world == 1 and not args.headline_only:
@@ -265,12 +281,22 @@ def run_native(args, rank, world, dev):
         "quantize_frac_hbm": round(q_gbs / pk["hbm_gbs"], 3),
         "gemm_tflops": round(gemm_tflops, 1),
         "frac_fp4_spec": round(value / world / FP4_SPEC_TFLOPS, 3),
+        "frac_fp4_incl_quantize": round(value / world / fp4_peak, 3),
         "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_pair_kernel<bf16>",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / fp4_peak, 3),
-                     "peak_src": f"{pk['src']} bf16 sustained x {FP4_OVER_BF16:g} (nominal fp4/bf16); "
-                                 f"burst peak {fp4_peak_burst:.1f} -> frac {gemm_tflops / fp4_peak_burst:.3f}",
+                     "peak_src": f"{pk['src']} bf16 {peak_kind} x {FP4_OVER_BF16:g} (nominal fp4/bf16), "
+                                 f"chosen from the sampled clocks (sustained only when sw_power_cap held "
+                                 f"most samples); burst {fp4_peak_burst:.1f} -> frac "
+                                 f"{gemm_tflops / fp4_peak_burst:.3f}, sustained {fp4_peak_sust:.1f} -> frac "
+                                 f"{gemm_tflops / fp4_peak_sust:.3f}, NVIDIA dense spec {FP4_SPEC_TFLOPS:.0f} -> "
+                                 f"frac {gemm_tflops / FP4_SPEC_TFLOPS:.3f}",
                      "traffic": recorded_traffic("gemm_prefill_mlp_gate_up")},
+        "roofline_quant": {"bound": "hbm", "kernel": "quantize_tma_kernel<bf16>",
+                           "achieved": round(q_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": round(q_gbs / pk["hbm_gbs"], 3),
+                           "per_unit": "2 B read + 0.5 B codes + 1/16 B scale per element",
+                           "traffic": recorded_traffic("quantize_prefill_mlp_gate_up", QUANT_SOURCES)},
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clocks,
@@ -280,7 +306,7 @@ def run_native(args, rank, world, dev):
     return out
 
 
-def measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world, steps=3):
+def measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world, steps=20):
     """Same metric through w4a4_gemm with host buffers: pinned H2D of X, the
     layer, D2H of Y, all inside the timed region."""
     x_host = x_cpu.pin_memory()
@@ -307,7 +333,7 @@ def measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world, steps
     ms = max_over_ranks([ms], world, dev)[0]
     del ws, x_dev, y_dev
     return {"value": round(job_throughput(2.0 * M * N * K, world, ms), 2), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": x_host.numel() * 2,
+            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": x_host.numel() * 2,
             "d2h_bytes_per_step": y_host.numel() * 2}
 
 

@@ -40,7 +40,7 @@
  *   - The caller allocates every buffer (PyTorch in the bundled binding); the
  *     library never calls cudaMalloc/cudaFree.
  *   - All work is enqueued on `stream`; nothing synchronizes the host except
- *     nvfp4_last_device_status().
+ *     nvfp4_last_device_status(), which synchronizes the stream it is given.
  *   - Preconditions: K % 64 == 0, K > 0, rows >= 0; device pointers 16-byte
  *     aligned; ld_x >= K with ld_x * element size a multiple of 16 bytes;
  *     ld_y >= N (any value); inputs finite; global scales finite and > 0.
@@ -201,8 +201,12 @@ nvfp4_status w4a4_gemm(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const f
  * mean what they mean for w4a4_gemm; the caller still provides x, the
  * weights, the scales and y.
  *   - Problems whose w4a4_gemm_workspace_bytes(M, N, K) exceeds 8 MiB return
- *     NVFP4_ERR_SCRATCH_LIMIT before anything is enqueued (decode-shaped
- *     products, e.g. M <= 64 with N*K up to about 5120 x 17408, fit).
+ *     NVFP4_ERR_SCRATCH_LIMIT before anything is enqueued.  That size is what
+ *     decides; as an example, on a B200 (where narrow products reduce inside a
+ *     thread-block cluster and need no partial sums) the decode products with
+ *     M <= 64 and N*K up to 5120 x 17408 fit, while on a device without
+ *     cluster support the same M = 64 products need split-K partial sums and
+ *     can exceed the buffer.
  *   - The first call on a device looks the buffer's device address up
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture on the device.
@@ -235,8 +239,8 @@ nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, c
 /*
  * Failure-detection self-test: launches one thread that waits, bounded by
  * limit_ns of %globaltimer (0 < limit_ns <= 2e9), on a barrier nothing ever
- * completes.  The wait runs out, sets bit 16 of the device error word (read
- * and cleared by nvfp4_last_device_status, which then returns
+ * completes.  The wait runs out, sets bit 4 (value 16) of the device error
+ * word (read and cleared by nvfp4_last_device_status, which then returns
  * NVFP4_ERR_TIMEOUT) and writes 0 to *result_dev (device int); the kernel
  * returns normally and the context stays usable.  Every wait in the library's
  * kernels is bounded the same way (2 s), so a lost producer or consumer shows
@@ -365,13 +369,23 @@ nvfp4_status nvfp4_plan_for(int64_t M, int64_t N, int64_t K, int sms, int pair_c
                             const int *split_clusters, int *out);
 
 /*
- * Synchronizes the device, then reports and clears the library's device error
- * word: *flags receives the OR of the flags kernels recorded since the last
- * call (bit 0: a producer wait ran out, bit 1: an MMA wait ran out, bit 2: an
- * epilogue wait ran out, bit 3: a TMEM allocation wait ran out).  Returns
- * NVFP4_ERR_TIMEOUT if any flag was set, NVFP4_ERR_CUDA on a CUDA error.
+ * Reports and clears the library's device error word of the current device:
+ * a one-thread kernel enqueued on `stream` takes the word and zeroes it in one
+ * atomic exchange, then this call synchronizes `stream` only (not the whole
+ * device) and stores the taken word in *flags (host int).  The word is the OR
+ * of the flags recorded by every library kernel that finished before that
+ * exchange, on any stream (flags of kernels still running on other streams
+ * are kept for the next call):
+ *   bit 0 (1)  : a producer wait ran out
+ *   bit 1 (2)  : an MMA-issue wait ran out
+ *   bit 2 (4)  : an epilogue or encoder wait ran out
+ *   bit 3 (8)  : a TMEM allocation wait ran out
+ *   bit 4 (16) : the self-test's wait ran out (nvfp4_selftest_wait_timeout)
+ * Returns NVFP4_ERR_TIMEOUT if any flag was set, NVFP4_ERR_CUDA on a CUDA
+ * error (including an earlier asynchronous fault that the synchronization
+ * surfaces), NVFP4_ERR_UNSUPPORTED on a device that is not sm_100.
  */
-nvfp4_status nvfp4_last_device_status(int *flags);
+nvfp4_status nvfp4_last_device_status(nvfp4_stream_t stream, int *flags);
 
 /* Static string for a status code. */
 const char *nvfp4_status_string(nvfp4_status status);

@@ -21,6 +21,7 @@
 using namespace nvfp4;
 
 __device__ unsigned g_nvfp4_device_error;
+__device__ unsigned g_nvfp4_error_snapshot;   // the word as nvfp4_last_device_status took it
 
 // Fixed scratch of w4a4_gemm_noalloc (see the header): quantized activation
 // and split-K partial sums for callers that cannot allocate.
@@ -649,8 +650,6 @@ nvfp4_status quantize_impl(const void *x, nvfp4_in_dtype dt, int64_t rows, int64
                              : launch_quantize<float>(p, *dev, s, pdl);
 }
 
-constexpr unsigned ERR_SELFTEST = 16u;   // error-word bit of the self-test below
-
 // mbar_wait with a caller-chosen limit (the self-test of the timeout path).
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, unsigned *err, unsigned code,
                                                 unsigned long long limit_ns) {
@@ -677,6 +676,9 @@ __global__ void wait_timeout_selftest_kernel(unsigned *err, unsigned long long l
     *result = ok ? 1 : 0;
   }
 }
+
+// Reads and clears the error word in one atomic exchange.
+__global__ void error_take_kernel(unsigned *err) { g_nvfp4_error_snapshot = atomicExch(err, 0u); }
 
 }  // namespace
 
@@ -817,6 +819,10 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
   if (x_dt != NVFP4_IN_BF16 && x_dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
   if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ld_x < K) return NVFP4_ERR_SHAPE;
   if (M == 0 || N == 0) return NVFP4_OK;
+  // the device checks first, so that an unsupported GPU reports UNSUPPORTED
+  DeviceState *state = nullptr;
+  nvfp4_status st = device_state(&state);
+  if (st != NVFP4_OK) return st;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
   void *buf = nullptr;
@@ -824,7 +830,10 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
     std::lock_guard<std::mutex> lock(mu);
     if (!scratch[dev]) {
       void *p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NVFP4_ERR_CUDA;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();      // leave no stale error for the next call's launch check
+        return NVFP4_ERR_CUDA;
+      }
       scratch[dev] = p;
     }
     buf = scratch[dev];
@@ -1041,13 +1050,21 @@ nvfp4_status nvfp4_selftest_wait_timeout(int64_t limit_ns, int *result_dev, nvfp
   return launched();
 }
 
-nvfp4_status nvfp4_last_device_status(int *flags) {
+nvfp4_status nvfp4_last_device_status(nvfp4_stream_t stream, int *flags) {
   if (!flags) return NVFP4_ERR_NULL;
   *flags = 0;
-  if (cudaDeviceSynchronize() != cudaSuccess) return NVFP4_ERR_CUDA;
-  unsigned v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, g_nvfp4_device_error, sizeof(v)) != cudaSuccess) return NVFP4_ERR_CUDA;
-  if (cudaMemcpyToSymbol(g_nvfp4_device_error, &zero, sizeof(zero)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  DeviceState *dev = nullptr;
+  nvfp4_status st = device_state(&dev);
+  if (st != NVFP4_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // take the word and clear it in one atomic step on the stream, so a flag
+  // that a kernel on another stream sets meanwhile is never lost
+  error_take_kernel<<<1, 1, 0, s>>>(dev->err);
+  if (launched() != NVFP4_OK) return NVFP4_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_nvfp4_error_snapshot, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
   *flags = (int)v;
   return v ? NVFP4_ERR_TIMEOUT : NVFP4_OK;
 }

@@ -10,7 +10,7 @@
 namespace nvfp4 {
 
 // error-word bits (reported by nvfp4_last_device_status)
-enum : unsigned { ERR_PRODUCER = 1u, ERR_MMA = 2u, ERR_EPILOGUE = 4u, ERR_TMEM = 8u };
+enum : unsigned { ERR_PRODUCER = 1u, ERR_MMA = 2u, ERR_EPILOGUE = 4u, ERR_TMEM = 8u, ERR_SELFTEST = 16u };
 
 // a single wait gives up after this many nanoseconds of %globaltimer
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -55,7 +55,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_rmsnorm_quantize.argtypes = [vp, i32, i64, i64, i64, vp, i32, ctypes.c_float, vp, vp, vp, vp, vp]
         L.nvfp4_selftest_wait_timeout.argtypes = [i64, vp, vp]
         L.nvfp4_plan_for.argtypes = [i64, i64, i64, i32, i32, vp, vp]
-        L.nvfp4_last_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.nvfp4_last_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_launch_count.argtypes, L.nvfp4_launch_count.restype = [], ctypes.c_uint64
         for f in ("nvfp4_amax_gscale", "nvfp4_quantize", "nvfp4_harmonize_group", "nvfp4_gemm",
@@ -438,9 +438,10 @@ def selftest_wait_timeout(limit_ns: int = 50_000_000) -> torch.Tensor:
 
 
 def last_device_status() -> int:
-    """Synchronize, then return and clear the device error flags (0 = clean)."""
+    """Take and clear the device error flags on the current stream, wait for
+    that stream, and return the flags (0 = clean)."""
     flags = ctypes.c_int(0)
-    st = lib().nvfp4_last_device_status(ctypes.byref(flags))
+    st = lib().nvfp4_last_device_status(_stream(), ctypes.byref(flags))
     if st not in (0, 6):
         raise Nvfp4Error("nvfp4_last_device_status", st)
     return flags.value

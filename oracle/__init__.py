@@ -12,8 +12,10 @@ Quantization"): the NVFP4 format and the W4A4 product on the ta-paperlens page
 ("前提1") and the arxiv-wiki page ("접근 방법"); the fused-group global-scale
 repair on the arxiv-wiki page ("접근 방법", "개발자 관점") and the abstract on the
 shd-paper page.  Readings the pages leave open are listed in the C file's
-header.  Everything except the arithmetic order for non-power-of-two global
-scales is pinned by tests/test_oracle_*.py; that order is "parity unpinned".
+header.  Every step is pinned by tests/test_oracle_*.py; the arithmetic order
+for non-power-of-two global scales (a reading: the pages do not fix it) is
+pinned against an exact rational evaluation of that reading on inputs at the
+rounding boundaries, where other orders give different bytes.
 The rows marked "next" (GDN gate activations, fake-quant, FP8 KV quantize,
 the re-quantizing harmonize and the quantize fused into the preceding
 RMSNorm) follow the same pages (ta-paperlens "前提2": the GDN layer feeds the

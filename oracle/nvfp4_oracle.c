@@ -32,11 +32,13 @@
  * least significant bit is 0 wins; a magnitude beyond the largest finite
  * value maps to that value (satfinite).
  *
- * Parity pins live in tests/test_oracle_*.py.  The arithmetic-order reading
- * (6*g first, true division) is not fixed by the pages: for power-of-two
- * global scales every order agrees and the round-trip pin covers it; for other
- * global scales the order is this file's reading ("parity unpinned" for the
- * order itself; the encoders and the layout are pinned).
+ * Parity pins live in tests/test_oracle_*.py.  The arithmetic order (6*g
+ * first, true division by d) is a reading, since the pages do not fix it; the
+ * pins hold this file to that reading at non-power-of-two global scales: an
+ * exact rational evaluation of the steps above, rounded to binary32 after
+ * each one, on inputs a few ulps from the E4M3 midpoints and the E2M1
+ * decision boundaries, where the other plausible orders (amax/6/g, x*(1/d),
+ * x/dec(s)/g) give different bytes.
  */
 #include <math.h>
 #include <stdint.h>

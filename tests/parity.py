@@ -67,8 +67,18 @@ def assert_gemm_close(y_gpu: torch.Tensor, y_ref: np.ndarray, yabs: np.ndarray):
     return float(np.max(err / np.maximum(yabs, 1e-300)))
 
 
-def gpu_gscale(x: torch.Tensor) -> torch.Tensor:
-    return native.amax_gscale(x)
+def checked_gscale(x_cpu: torch.Tensor, x_dev: torch.Tensor | None = None):
+    """The global scale of an input as the oracle computes it on the CPU copy,
+    checked bit for bit against the library's nvfp4_amax_gscale on the device
+    copy.  Returns (the oracle's value as np.float32, the same value as a
+    1-element device tensor): both sides of a parity test then start from the
+    oracle's scale, and no oracle input comes from the CUDA path."""
+    g_ref = oracle.global_scale(to_f32_numpy(x_cpu))
+    if x_dev is None:
+        x_dev = x_cpu.to("cuda")
+    g_gpu = f32(native.amax_gscale(x_dev))
+    assert np.array([g_gpu]).view(np.uint32)[0] == np.array([g_ref]).view(np.uint32)[0], (g_gpu, g_ref)
+    return g_ref, torch.tensor([g_ref], dtype=torch.float32, device=x_dev.device)
 
 
 def f32(t: torch.Tensor) -> np.float32:

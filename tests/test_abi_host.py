@@ -139,3 +139,23 @@ def test_requant_and_rmsnorm_validation(L):
     assert r(FAKE, 1, 4, 23232, 23232, FAKE, 0, 1e-6, *tail) == 5
     assert r(FAKE, 0, 4, 38592, 38592, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
     assert r(FAKE, 1, 4, 23168, 23168, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
+
+
+def test_error_word_bits_match_the_header(L):
+    """The flag values nvfp4_last_device_status documents are the values the
+    kernels OR into the device error word."""
+    src = os.path.join(os.path.dirname(HEADER), "..", "nvfp4_w4a4_quantized_06_b200", "csrc", "ptx.cuh")
+    enum = re.search(r"enum\s*:\s*unsigned\s*\{([^}]*)\}", open(src).read()).group(1)
+    code_bits = {n: int(v) for n, v in re.findall(r"(ERR_[A-Z]+)\s*=\s*(\d+)u", enum)}
+    assert code_bits == {"ERR_PRODUCER": 1, "ERR_MMA": 2, "ERR_EPILOGUE": 4, "ERR_TMEM": 8, "ERR_SELFTEST": 16}
+    doc = open(HEADER).read()
+    block = doc[doc.index("Reports and clears the library's device error word"):doc.index("nvfp4_last_device_status(nvfp4_stream_t")]
+    listed = {int(b): int(v) for b, v in re.findall(r"bit (\d+) \((\d+)\)", block)}
+    assert listed == {0: 1, 1: 2, 2: 4, 3: 8, 4: 16}
+    assert set(listed.values()) == set(code_bits.values())
+    assert "bit 4 (value 16)" in doc[doc.index("Failure-detection self-test"):]
+
+
+def test_last_device_status_takes_a_stream(L):
+    assert L.nvfp4_last_device_status.argtypes[0] is ctypes.c_void_p
+    assert L.nvfp4_last_device_status(None, None) == 1                       # null flags: rejected first

@@ -8,7 +8,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_06_b200 import native
 from nvfp4_w4a4_quantized_06_b200 import workloads as W
-from parity import assert_codes_equal, assert_gemm_close, f32, to_f32_numpy
+from parity import assert_codes_equal, assert_gemm_close, checked_gscale, f32, to_f32_numpy
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -25,7 +25,7 @@ def _quantized_weight(wl):
     for m in range(len(wl.modules)):
         w = W.make_w(wl, m)
         wd = w.to(DEV)
-        g = native.amax_gscale(wd)
+        _, g = checked_gscale(w, wd)
         native.quantize(wd, g, codes=codes[offs[m]:offs[m + 1]], sf=sf, sf_row0=int(offs[m]), sf_rows_total=N)
         mods.append((w, g))
     if len(mods) > 1:
@@ -61,7 +61,7 @@ def _oracle_weight_rows(wl, mods, offs, cols):
 def _run_linear(wl, out_dtype, rows=None, cols=None):
     x_cpu = W.make_x(wl)
     x = x_cpu.to(DEV)
-    gx = native.amax_gscale(x)
+    _, gx = checked_gscale(x_cpu, x)
     codes, sf, gw, mods, offs = _quantized_weight(wl)
     y = native.linear(x, gx, codes, sf, gw, out_dtype=out_dtype)
     torch.cuda.synchronize()
@@ -85,7 +85,7 @@ def _random_case(M, N, K, seed, out_dtype, a_dtype=torch.bfloat16):
     x_cpu = W.gaussian(M, K, seed=seed, outliers=W.Outliers("scale", 0.02, 30.0), dtype=a_dtype)
     w_cpu = W.gaussian(N, K, seed=seed + 1, std=0.02, dtype=a_dtype)
     x, w = x_cpu.to(DEV), w_cpu.to(DEV)
-    gx, gw = native.amax_gscale(x), native.amax_gscale(w)
+    (_, gx), (_, gw) = checked_gscale(x_cpu, x), checked_gscale(w_cpu, w)
     ac, asf = native.quantize(x, gx)
     bc, bsf = native.quantize(w, gw)
     y = native.gemm(ac, asf, gx, bc, bsf, gw, out_dtype=out_dtype)
@@ -126,7 +126,7 @@ def test_gemm_pair_shapes(M, N, K, out_dtype):
     x_cpu = W.gaussian(M, K, seed=M, outliers=W.Outliers("scale", 0.02, 30.0))
     w_cpu = W.gaussian(N, K, seed=N, std=0.02)
     x, w = x_cpu.to(DEV), w_cpu.to(DEV)
-    gx, gw = native.amax_gscale(x), native.amax_gscale(w)
+    (_, gx), (_, gw) = checked_gscale(x_cpu, x), checked_gscale(w_cpu, w)
     ac, asf = native.quantize(x, gx)
     bc, bsf = native.quantize(w, gw)
     y = native.gemm(ac, asf, gx, bc, bsf, gw, out_dtype=out_dtype)
@@ -151,14 +151,18 @@ def test_gemm_fp32_activation():
     _random_case(96, 128, 512, seed=5, out_dtype=torch.float32, a_dtype=torch.float32)
 
 
-def test_gdn_gates_fused_group():
-    _run_linear(W.WORKLOADS["gdn_gates_ab"], torch.float32, rows=W.sample_rows(4096, 512))
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gdn_gates_fused_group(out_dtype):
+    """The whole 4096 x 96 x 5120 gate product, every output checked."""
+    _run_linear(W.WORKLOADS["gdn_gates_ab"], out_dtype)
 
 
 @pytest.mark.parametrize("name", ["decode_out_proj", "decode_down_proj"])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_decode_workloads(name, out_dtype):
-    _run_linear(W.WORKLOADS[name], out_dtype, cols=W.sample_rows(5120, 640))
+    """The whole decode product (32 x 5120 x 5120 or 32 x 5120 x 17408), every
+    output checked."""
+    _run_linear(W.WORKLOADS[name], out_dtype)
 
 
 def test_gdn_qkv_z_fused_group():
@@ -184,15 +188,21 @@ def test_prefill_mlp_full_size():
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_fused_prologue_matches_layer(M, N, K, x_dtype, out_dtype):
     """The in-GEMM activation quantize gives the two-kernel layer's output bit
-    for bit (same codes, same MMAs, same reduction order)."""
-    x = W.gaussian(M, K, seed=M + 3, outliers=W.Outliers("scale", 0.02, 30.0), dtype=x_dtype).to(DEV)
-    w = W.gaussian(N, K, seed=N + 5, std=0.02).to(DEV)
-    gx, gw = native.amax_gscale(x), native.amax_gscale(w)
+    for bit (same codes, same MMAs, same reduction order), and both are within
+    the GEMM tolerance of the oracle's float64 reference."""
+    x_cpu = W.gaussian(M, K, seed=M + 3, outliers=W.Outliers("scale", 0.02, 30.0), dtype=x_dtype)
+    w_cpu = W.gaussian(N, K, seed=N + 5, std=0.02)
+    x, w = x_cpu.to(DEV), w_cpu.to(DEV)
+    (gx_r, gx), (gw_r, gw) = checked_gscale(x_cpu, x), checked_gscale(w_cpu, w)
     wc, ws = native.quantize(w, gw)
     y_ref = native.linear(x, gx, wc, ws, gw, out_dtype=out_dtype)
     y = native.linear_fused(x, gx, wc, ws, gw, out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert native.last_device_status() == 0
+    rwc, rws = oracle.quantize(to_f32_numpy(w_cpu), gw_r)
+    assert_codes_equal(wc, rwc)
+    y64, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu), gx_r, rwc, rws, gw_r)
+    assert_gemm_close(y, y64, yabs)
     assert torch.equal(y, y_ref)
 
 

@@ -9,7 +9,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_06_b200 import native
 from nvfp4_w4a4_quantized_06_b200 import workloads as W
-from parity import assert_codes_equal, assert_sf_rows_equal, f32, to_f32_numpy
+from parity import assert_codes_equal, assert_sf_rows_equal, checked_gscale, f32, to_f32_numpy
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -24,7 +24,7 @@ def _gate_weights(wl):
     mods = []
     for m in range(len(wl.modules)):
         w = W.make_w(wl, m)
-        g = native.amax_gscale(w.to(DEV))
+        _, g = checked_gscale(w)
         native.quantize(w.to(DEV), g, codes=codes[offs[m]:offs[m + 1]], sf=sf, sf_row0=int(offs[m]), sf_rows_total=N)
         mods.append((w, g))
     gstar = native.harmonize(sf, N, K, offs, torch.cat([g for _, g in mods]))
@@ -42,21 +42,20 @@ def _gate_weights(wl):
 @pytest.mark.parametrize("M", [4096, 32])
 def test_gdn_gates_fused_epilogue(M):
     """alpha = exp(-softplus(a)) on the 48 a columns, beta = sigmoid(b) on the
-    48 b columns.  Both activations have slope at most 1/4, so the bound is a
+    48 b columns, every output of the launch checked.  Both activations have slope at most 1/4, so the bound is a
     quarter of the GEMM's 1e-3 * sum|products|, plus the fp32 evaluation of
     exp / log1p (a few ulps of values <= 1)."""
     wl = W.WORKLOADS["gdn_gates_ab"]
     codes, sf, gw, rcodes, rsf, rg = _gate_weights(wl)
     x_cpu = W.make_x(wl)[:M]
     x = x_cpu.to(DEV)
-    gx = native.amax_gscale(x)
+    _, gx = checked_gscale(x_cpu, x)
     out = native.gdn_gates(x, gx, codes, sf, gw, n_a=wl.modules[0])
     torch.cuda.synchronize()
     assert native.last_device_status() == 0
-    rows = W.sample_rows(M, min(M, 384), seed=5)
-    y_ref, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu[torch.from_numpy(rows)]), f32(gx), rcodes, rsf, rg)
+    y_ref, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu), f32(gx), rcodes, rsf, rg)
     ref = oracle.gdn_gates(y_ref, wl.modules[0])
-    got = out[torch.from_numpy(rows).to(DEV)].double().cpu().numpy()
+    got = out.double().cpu().numpy()
     tol = 0.25 * GEMM_RTOL * yabs + 1e-5 * np.abs(ref) + 1e-7
     err = np.abs(got - ref)
     assert np.all(err <= tol), float((err - tol).max())
@@ -69,11 +68,11 @@ def test_gdn_gates_fused_epilogue(M):
 def test_fake_quant_bit_exact(rows, K, in_dtype, out_dtype):
     x_cpu = W.gaussian(rows, K, seed=rows + K, outliers=W.Outliers("scale", 0.03, 35.0), dtype=in_dtype)
     x = x_cpu.to(DEV)
-    g = native.amax_gscale(x)
+    g_ref, g = checked_gscale(x_cpu, x)
     out, stats = native.fake_quant(x, g, out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert native.last_device_status() == 0
-    dq, se, sx = oracle.fake_quant(to_f32_numpy(x_cpu), f32(g))
+    dq, se, sx = oracle.fake_quant(to_f32_numpy(x_cpu), g_ref)
     ref = torch.from_numpy(dq.astype(np.float32)).to(out_dtype)       # exact value rounded to fp32, then to bf16
     assert torch.equal(out.cpu(), ref)
     st = stats.cpu().numpy()
@@ -216,12 +215,12 @@ def _check_rmsnorm(x_cpu, w_cpu, eps, zero_centered, rows=None):
     rc, rs, _, rinv, near = oracle.rmsnorm_quantize(xs, wn, eps, g, zero_centered)
     torch.cuda.synchronize()
     ginv = inv.cpu().numpy()[sel]
-    if near.any():
-        # the exact factor sits within ~2^-45 of a rounding midpoint: either
-        # neighbour is acceptable, and the codes must follow the one chosen
-        idx = np.flatnonzero(near)
-        assert np.all(np.abs(ginv[idx].view(np.int32) - rinv[idx].view(np.int32)) <= 1)
-        rc, rs, _, rinv, _ = oracle.rmsnorm_quantize(xs, wn, eps, g, zero_centered, inv=ginv)
+    # The kernel evaluates the mean square to about 2^-48 relative, so it
+    # rounds the per-row factor correctly unless the exact value lies within
+    # ~2^-45 of a midpoint between two floats; the oracle flags such rows.
+    # The seeded inputs are chosen so that no row is that close: every row is
+    # then compared with the oracle's correctly rounded factor, bit for bit.
+    assert not near.any(), f"rows {np.flatnonzero(near)} sit at a rounding midpoint; change the seed"
     assert np.array_equal(ginv.view(np.uint32), rinv.view(np.uint32)), "per-row factor differs"
     if rows is None:
         assert_codes_equal(codes, rc)

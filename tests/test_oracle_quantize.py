@@ -242,3 +242,161 @@ def test_unharmonized_fused_gemm_shows_scale_mismatch(oracle):
     gstar = oracle.harmonize(sf, K, offs, gs)
     fixed = oracle.dequantize(codes, sf, gstar)
     assert np.linalg.norm(fixed - right) / np.linalg.norm(right) < 2 ** -4
+
+
+# ------------------------------------------------ arithmetic order, exactly
+# The pages fix the block scale as "block maximum / 6" relative to a per-tensor
+# FP32 scale (ta-paperlens page, 前提1) but not the order of the fp32 steps.
+# The reading the oracle states is
+#   g6 = fl32(6 g), t = fl32(amax / g6), s = E4M3(t), d = fl32(dec(s) g), y = fl32(x / d).
+# The checks below evaluate that reading in exact rational arithmetic, with an
+# explicit round-to-nearest-even onto binary32 after each step, at global
+# scales that are not powers of two, on inputs placed within a few ulps of the
+# E4M3 midpoints and the E2M1 decision boundaries, where a different order of
+# operations changes the result.
+from fractions import Fraction as Fr  # noqa: E402
+
+E2M1_MAG = [Fr(0), Fr(1, 2), Fr(1), Fr(3, 2), Fr(2), Fr(3), Fr(4), Fr(6)]
+
+
+def _e4m3_mag(c):
+    e, m = c >> 3, c & 7
+    return Fr(m, 512) if e == 0 else (1 + Fr(m, 8)) * Fr(2) ** (e - 7)
+
+
+E4M3_MAG = [_e4m3_mag(c) for c in range(0x7F)]          # codes 0 .. 0x7E (448)
+
+
+def _fl32(q: Fr) -> Fr:
+    """The binary32 value nearest to the rational q (ties to even), subnormals
+    included; |q| stays far below the overflow threshold in these tests."""
+    if q == 0:
+        return Fr(0)
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fr(2) ** e > a:
+        e -= 1
+    while Fr(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fr(2) ** (max(e, -126) - 23)
+    m = a / quantum
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fr(1, 2) or (rem == Fr(1, 2) and n % 2 == 1):
+        n += 1
+    return (n * quantum) if q > 0 else -(n * quantum)
+
+
+def _nearest(a: Fr, grid):
+    """Index of the grid magnitude nearest to a >= 0; ties to the even index;
+    beyond the top the top index (satfinite)."""
+    if a >= grid[-1]:
+        return len(grid) - 1
+    best = 0
+    for c in range(1, len(grid)):
+        d, db = abs(a - grid[c]), abs(a - grid[best])
+        if d < db or (d == db and c % 2 == 0):
+            best = c
+    return best
+
+
+def _exact_block(xb, g, order="reading"):
+    """Scale byte and 16 codes of one block by the stated reading (or by one of
+    the plausible wrong orders, which the test shows the inputs can tell apart)."""
+    g = Fr(float(g))
+    xs = [Fr(float(v)) for v in xb]
+    amax = max(abs(v) for v in xs)
+    if order == "amax/6/g":
+        t = _fl32(_fl32(amax / 6) / g)
+    elif order == "6g exact":
+        t = _fl32(amax / (6 * g))
+    else:
+        t = _fl32(amax / _fl32(6 * g))
+    s = _nearest(t, E4M3_MAG)
+    decs = E4M3_MAG[s]
+    if decs == 0:
+        return s, [0] * 16
+    d = _fl32(decs * g)
+    codes = []
+    for v in xs:
+        if order == "x*(1/d)":
+            y = _fl32(v * _fl32(1 / d))
+        elif order == "x/dec(s)/g":
+            y = _fl32(_fl32(v / decs) / g)
+        else:
+            y = _fl32(v / d)
+        c = _nearest(abs(y), E2M1_MAG)
+        codes.append(c | (8 if y < 0 or (y == 0 and v < 0) else 0))
+    return s, codes
+
+
+def _ulps(v: np.float32, k: int) -> np.float32:
+    return (np.array([v], np.float32).view(np.int32) + k).view(np.float32)[0]
+
+
+def _order_probe_blocks(g: np.float32) -> np.ndarray:
+    """Blocks whose maximum lands within 3 ulps of an E4M3 midpoint (after the
+    division by fl32(6g)), and blocks whose other 15 elements land within 2
+    ulps of an E2M1 decision boundary (after the division by d)."""
+    g6 = np.float32(6) * g
+    blocks = []
+    mids = [(E4M3_MAG[c] + E4M3_MAG[c + 1]) / 2 for c in range(8, 0x7E, 5)]     # normal range
+    for mid in mids:
+        centre = np.float32(float(mid) * float(g6))
+        for k in range(-3, 4):
+            b = np.zeros(16, np.float32)
+            b[0] = _ulps(centre, k)
+            b[1:] = b[0] * np.float32(0.25)
+            blocks.append(b)
+    bounds = [Fr(1, 4), Fr(3, 4), Fr(5, 4), Fr(7, 4), Fr(5, 2), Fr(7, 2), Fr(5)]
+    for sc in (0x2B, 0x3D, 0x46, 0x59, 0x6A):                # scale codes to aim at
+        amax = np.float32(6 * float(E4M3_MAG[sc]) * float(g6))
+        decs = Fr(float(E4M3_MAG[_nearest(_fl32(Fr(float(amax)) / _fl32(6 * Fr(float(g)))), E4M3_MAG)]))
+        d = _fl32(decs * Fr(float(g)))
+        vals = [np.float32(float(T * d)) for T in bounds]
+        probes = [_ulps(v, k) for v in vals for k in (-2, -1, 0, 1, 2)]
+        for i in range(0, len(probes), 15):
+            b = np.zeros(16, np.float32)
+            b[0] = amax
+            chunk = probes[i:i + 15]
+            b[1:1 + len(chunk)] = [p if j % 2 else -p for j, p in enumerate(chunk)]
+            blocks.append(b)
+    n = len(blocks) + (-len(blocks)) % 4                     # whole 64-element rows
+    blocks += [np.zeros(16, np.float32)] * (n - len(blocks))
+    return np.stack(blocks).reshape(-1, 64)
+
+
+ORDER_GSCALES = [np.float32(0.37 / 2688), np.float32(3.3 / 2688), np.float32(0.0123), np.float32(0.7 / 2688)]
+
+
+def test_arithmetic_order_matches_the_exact_reading(oracle):
+    detected = {alt: 0 for alt in ("amax/6/g", "x*(1/d)", "x/dec(s)/g", "6g exact")}
+    for g in ORDER_GSCALES:
+        x = _order_probe_blocks(g)
+        rows = x.shape[0]
+        codes, sf = oracle.quantize(x, g)
+        got_s = oracle.sf_gather(sf, np.arange(rows), 64).reshape(-1)
+        got_q = np.stack([codes & 15, codes >> 4], axis=-1).reshape(-1, 16)
+        blocks = x.reshape(-1, 16)
+        want = [_exact_block(b, g) for b in blocks]
+        for i, (s, q) in enumerate(want):
+            assert got_s[i] == s, (float(g), i, got_s[i], s)
+            assert list(got_q[i]) == q, (float(g), i, list(got_q[i]), q)
+        for alt in detected:
+            detected[alt] += sum(_exact_block(b, g, alt) != w for b, w in zip(blocks, want))
+    # the probes are sharp enough to tell the stated order from the plausible
+    # alternatives: each of them changes scales or codes on these inputs
+    assert all(n > 0 for n in detected.values()), detected
+
+
+def test_exact_reading_helpers():
+    """The rational helpers against plain facts: binary32 rounding at a tie,
+    a subnormal, and the E4M3 / E2M1 grids' ends and ties."""
+    assert _fl32(Fr(1) + Fr(2) ** -24) == 1                          # tie -> even
+    assert _fl32(Fr(1) + Fr(3, 2 ** 25)) == 1 + Fr(2) ** -23          # above the tie
+    assert _fl32(Fr(3, 2 ** 151)) == Fr(1, 2 ** 149)                  # subnormal quantum
+    assert _fl32(Fr(1, 3)) == Fr(float(np.float32(1 / 3)))
+    assert _nearest(Fr(1, 4), E2M1_MAG) == 0 and _nearest(Fr(3, 4), E2M1_MAG) == 2
+    assert _nearest(Fr(5), E2M1_MAG) == 6 and _nearest(Fr(100), E2M1_MAG) == 7
+    assert E4M3_MAG[0x7E] == 448 and E4M3_MAG[1] == Fr(1, 512) and E4M3_MAG[8] == Fr(1, 64)
+    assert _nearest(Fr(17, 16), E4M3_MAG) == 0x38                     # 1.0625: tie -> 1.0 (even)

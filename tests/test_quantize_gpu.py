@@ -7,7 +7,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_06_b200 import native
 from nvfp4_w4a4_quantized_06_b200 import workloads as W
-from parity import assert_codes_equal, assert_sf_rows_equal, f32, to_f32_numpy
+from parity import assert_codes_equal, assert_sf_rows_equal, checked_gscale, f32, to_f32_numpy
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -122,7 +122,7 @@ def test_fused_group_offsets_and_padding():
     gs = []
     for i, (w, r0) in enumerate(((w0, 0), (w1, 48))):
         wd = w.to(DEV)
-        g = native.amax_gscale(wd)
+        _, g = checked_gscale(w, wd)
         gs.append(g)
         native.quantize(wd, g, codes=codes[r0:r0 + 48], sf=sf, sf_row0=r0, sf_rows_total=96)
     ref_sf = np.zeros(oracle.sf_bytes(96, K), np.uint8)
@@ -156,11 +156,9 @@ def test_workload_sampled_rows(name):
     tensors = [W.make_x(wl)] + [W.make_w(wl, m) for m in range(len(wl.modules))]
     for t in tensors:
         x = t.to(DEV)
-        g = native.amax_gscale(x)
+        g_ref, g = checked_gscale(t, x)
         codes, sf = native.quantize(x, g)
         rows = W.sample_rows(t.shape[0], 192)
-        g_ref = oracle.global_scale(to_f32_numpy(t))
-        assert f32(g) == g_ref
         rc, rs = oracle.quantize(to_f32_numpy(t[torch.from_numpy(rows)]), g_ref)
         torch.cuda.synchronize()
         assert_codes_equal(codes[torch.from_numpy(rows).to(DEV)], rc)
@@ -186,7 +184,7 @@ def test_harmonize_workload_groups():
             w = W.make_w(wl, m)
             ws.append(w)
             wd = w.to(DEV)
-            g = native.amax_gscale(wd)
+            _, g = checked_gscale(w, wd)
             gs.append(g)
             native.quantize(wd, g, codes=codes[offs[m]:offs[m + 1]], sf=sf, sf_row0=int(offs[m]),
                             sf_rows_total=N)
