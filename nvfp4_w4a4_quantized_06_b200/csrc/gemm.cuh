@@ -58,6 +58,7 @@ struct GemmParams {
   int64_t ld_x;             //   its row stride (elements)
   const float *x_gscale;    //   its global scale (device)
   unsigned *err;
+  int tma_store;            // CTA-pair GEMM, BF16 out: store Y through its tensor map
 };
 
 template <int BN>

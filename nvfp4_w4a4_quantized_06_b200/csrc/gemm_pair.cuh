@@ -14,10 +14,17 @@
 // Scale factors reach TMEM through tcgen05.st, not tcgen05.cp: the NVFP4
 // scales of a 128 x 256 x 256 slice are 24 KB of replicated TMEM columns per
 // SM per stage, which the smem->TMEM copy path moves at ~40 B/clk (slower
-// than the MMAs that consume them), while eight "scale warps" (per TMEM lane
-// quarter one for the A scales and one for the B scales) store them from
-// registers at several hundred B/clk and leave the single MMA-issuing thread
-// nothing but MMAs.
+// than the MMAs that consume them; the whole GEMM measured 3.86 ms against
+// 2.43 ms when the MMA thread issued tcgen05.cp.cta_group::2 per K block),
+// while eight "scale warps" (per TMEM lane quarter one for the A scales and
+// one for the B scales) store them from registers at several hundred B/clk
+// and leave the single MMA-issuing thread nothing but MMAs.
+//
+// BF16 output leaves through TMA stores: each epilogue warp drains its
+// accumulator columns, hands TMEM back, converts to BF16 in a 32 x 32 staging
+// box in shared memory and one lane stores the box (2.47 ms against 2.97 ms
+// with per-lane 16-byte register stores, whose 32 rows per instruction
+// crowd the SM's path to L2 that the operand loads share).
 //
 // Warp roles per CTA: 0 producer (one lane), 1 TMEM allocation + MMA issue
 // (one lane of the leader), 2-5 A-scale warps and 6-9 B-scale warps (lane
@@ -29,6 +36,10 @@
 
 #include "gemm.cuh"
 #include "ptx.cuh"
+
+#ifndef NVFP4_Y_EVICT_FIRST
+#define NVFP4_Y_EVICT_FIRST false
+#endif
 
 namespace nvfp4 {
 
@@ -51,7 +62,11 @@ struct PairCfg {
   static constexpr int SFA_COL = BN;
   static constexpr int SFB_COL = BN + 16;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  // BF16 output staging: one 32-row x 32-column box (64-byte rows, 64-byte
+  // swizzle) per epilogue warp, stored to Y by TMA
+  static constexpr int STG_WARP_BYTES = 32 * 64;
+  static constexpr int STG_BYTES = EPI_WARPS * STG_WARP_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_BYTES + 256;
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                     ((uint32_t)(256 >> 4) << 24);
   static_assert(BN + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
@@ -62,7 +77,7 @@ template <int MODE>
 __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                            const __grid_constant__ CUtensorMap tmsfa, const __grid_constant__ CUtensorMap tmsfb,
-                           const GemmParams p) {
+                           const __grid_constant__ CUtensorMap tmy, const GemmParams p) {
   using C = PairCfg;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -70,7 +85,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   uint8_t *sB = sA + C::STAGES * C::A_BYTES;
   uint8_t *sSFA = sB + C::STAGES * C::B_BYTES;
   uint8_t *sSFB = sSFA + C::STAGES * C::SFA_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sSFB + C::STAGES * C::SFB_BYTES);
+  uint8_t *sStg = sSFB + C::STAGES * C::SFB_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sStg + C::STG_BYTES);
   uint64_t *full = bars;                        // leader: A/B of both CTAs + own scales
   uint64_t *sffull = bars + C::STAGES;          // peer: own scales
   uint64_t *sfready = bars + 2 * C::STAGES;     // leader: scales in both TMEMs (8 warps)
@@ -105,6 +121,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     prefetch_tmap(&tmb);
     prefetch_tmap(&tmsfa);
     prefetch_tmap(&tmsfb);
+    if (p.tma_store) prefetch_tmap(&tmy);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
@@ -282,7 +299,29 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty_leader);
-        if (i < p.rows_a) {
+        if (p.tma_store) {
+          // lane l writes row l of a 32 x 32 box, 16-byte chunk j at j ^ ((l / 2) % 4)
+          // (the 64-byte swizzle: conflict-free for eight lanes at a time), then
+          // one lane stores the box; rows and columns past Y are not written
+          const int row0 = ta * 256 + (int)rank * C::BM + q * 32;
+          uint8_t *stg = sStg + ew * C::STG_WARP_BYTES;
+          uint4 *dst = reinterpret_cast<uint4 *>(stg + lane * 64);
+#pragma unroll
+          for (int c = 0; c < C::EPI_COLS; c += 32) {
+            if (lane == 0) bulk_wait_read_all();        // the previous box has left the buffer
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j ^ ((lane >> 1) & 3)] = make_uint4(packed[c / 2 + 4 * j], packed[c / 2 + 4 * j + 1],
+                                                      packed[c / 2 + 4 * j + 2], packed[c / 2 + 4 * j + 3]);
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0 && row0 < p.rows_a && j0 + c < p.rows_b) {
+              tma_store_2d<NVFP4_Y_EVICT_FIRST>(&tmy, stg, j0 + c, row0);
+              bulk_commit_group();
+            }
+          }
+        } else if (i < p.rows_a) {
           __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out);
 #pragma unroll
           for (int c = 0; c < C::EPI_COLS; c += 8) {
@@ -318,6 +357,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         if (lane == 0) mbar_arrive_cluster(tempty_leader);
       }
     }
+    if (lane == 0) bulk_wait_all();                 // Y boxes written before the CTA ends
   }
 
   // teardown: the leader's MMAs write this CTA's TMEM and read its shared

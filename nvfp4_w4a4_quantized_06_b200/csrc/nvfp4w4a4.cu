@@ -210,6 +210,21 @@ bool make_sf_map(CUtensorMap *map, const void *sf, int64_t rows, int64_t K, int 
   return r == CUDA_SUCCESS;
 }
 
+// Y as bf16 [M][N] (row stride ld_y) for the CTA-pair GEMM's TMA stores: a
+// box of 32 columns (64 bytes) x 32 rows with the 64-byte swizzle the
+// epilogue writes its staging boxes in.  Needs a 16-byte-aligned y and a row
+// stride that is a multiple of 8 elements (16 bytes).
+bool make_y_map(CUtensorMap *map, void *y, int64_t M, int64_t N, int64_t ld_y) {
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld_y * 2)};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // GEMM plan: which kernel, which operand drives the 128-row MMA dimension,
 // the tile width, split-K and the grid.
 struct Plan {
@@ -456,10 +471,18 @@ nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float 
     p.out = y;
     p.out_si = ld_y;
     p.out_sj = 1;
-    CUtensorMap ma, mb, msa, msb;
+    CUtensorMap ma, mb, msa, msb, my;
     if (!make_codes_map(&ma, a_codes, M, K, 128) || !make_codes_map(&mb, b_codes, N, K, 128) ||
         !make_sf_map(&msa, a_sf, M, K, 1) || !make_sf_map(&msb, b_sf, N, K, 2))
       return NVFP4_ERR_CUDA;
+    // BF16 output goes out through TMA stores when Y's layout allows it (the
+    // register-store epilogue serves the rest, and FP32 output)
+    p.tma_store = y_dt == NVFP4_OUT_BF16 && aligned16(y) && ld_y % 8 == 0 ? 1 : 0;
+    if (p.tma_store) {
+      if (!make_y_map(&my, y, M, N, ld_y)) return NVFP4_ERR_CUDA;
+    } else {
+      my = ma;                       // unused
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -473,8 +496,8 @@ nvfp4_status gemm_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = y_dt == NVFP4_OUT_BF16
-                        ? cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_BF16>, ma, mb, msa, msb, p)
-                        : cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_F32>, ma, mb, msa, msb, p);
+                        ? cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_BF16>, ma, mb, msa, msb, my, p)
+                        : cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<OUT_F32>, ma, mb, msa, msb, my, p);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     return launched();
   }

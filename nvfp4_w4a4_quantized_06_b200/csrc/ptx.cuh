@@ -329,6 +329,33 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// 2D tiled store of a shared-memory box to global memory through the tensor
+// map (elements outside the tensor are not written); completes in this
+// thread's bulk async-group.  With evict_first the written lines are the
+// first candidates for eviction from L2, so an output stream does not push
+// the GEMM's operands out.
+template <bool EVICT_FIRST = false>
+__device__ __forceinline__ void tma_store_2d(const void *tmap, const void *smem_src, int32_t x, int32_t y) {
+  if constexpr (EVICT_FIRST) {
+    asm volatile(
+        "{\n\t.reg .b64 pol;\n\t"
+        "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], pol;\n\t}" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+        : "memory");
+  } else {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+  }
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every bulk store of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until every bulk store of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // order this thread's generic-proxy shared-memory writes before later
 // async-proxy reads of them (TMA stores, tcgen05.mma operand fetches)
 __device__ __forceinline__ void fence_proxy_async_shared() {

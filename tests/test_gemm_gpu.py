@@ -117,7 +117,8 @@ def test_gemm_shapes(M, N, K, out_dtype):
 
 
 @pytest.mark.parametrize("M,N,K", [
-    (4200, 4396, 1344),   # CTA-pair path: last row tile's second CTA past M, N and K tails
+    (4200, 4396, 1344),   # CTA-pair path: last row tile's second CTA past M, N and K tails (register stores)
+    (4200, 4392, 1344),   # the same raggedness with Y rows a multiple of 16 bytes (TMA stores)
     (2304, 2560, 5120),   # CTA-pair path, exact tiles
 ])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
