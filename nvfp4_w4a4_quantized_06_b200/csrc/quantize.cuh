@@ -117,9 +117,6 @@ __device__ __forceinline__ float to_f32(float f) { return f; }
 constexpr float kWidenLo = 0.999999523162841796875f;   // 1 - 2^-21
 constexpr float kWidenHi = 1.000000476837158203125f;   // 1 + 2^-21
 
-// rounding boundary between E2M1 magnitudes m and m + 1
-__constant__ float kE2m1Boundary[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
-
 struct EncodeConsts {
   float g, g6, rg;          // g, fl32(6g), fl32(1/g)
   float rg6_lo, rg6_hi;     // fl32(1/g6) widened down and up by 2^-21
@@ -150,21 +147,35 @@ __device__ __forceinline__ void fill_rcp_table(float *tab) {
 __device__ __noinline__ float div_rn_slow(float a, float b) { return __fdiv_rn(a, b); }
 
 // Sign of fl32(a / b) - T for a >= 0 and b > 0 normal, T > 0 a normal float
-// with a short significand (an E2M1 boundary or an E4M3 midpoint).  With h+
-// and h- half the float spacing above and below T, RNE gives fl32(a/b) > T
-// exactly when a/b > T + h+, and fl32(a/b) < T exactly when a/b < T - h-
-// (at either bound the tie goes to T, whose last significand bit is 0).
-// Compared as a vs (T +- h) * b in fp64: T +- h needs at most 26 significant
-// bits and b 24, so the product and the comparison are exact.
+// with at most five significant bits (an E2M1 boundary or an E4M3 midpoint).
+// With h+ and h- half the float spacing above and below T, RNE gives
+// fl32(a/b) > T exactly when a/b > T + h+, and fl32(a/b) < T exactly when
+// a/b < T - h- (at either bound the tie goes to T, whose last significand bit
+// is 0); that is, when D = a - T*b is above h+ * b or below -h- * b.  One FMA
+// gives D: T*b has at most 29 significant bits and a at most 24, so wherever
+// a/b lies within 2^-17 of T the exact difference is a multiple of
+// 2^(e - 28) below 2^(e - 16) (e the exponent of T*b), i.e. it fits in 24
+// bits and the FMA returns it exactly; farther from T the rounded D keeps its
+// sign and stays far from h+-*b, so the comparison still decides correctly.
+// h+-*b are exact (powers of two times b, far above the subnormal range for
+// the scales this library accepts).
 __device__ __forceinline__ int quotient_vs(float a, float b, float T) {
   const uint32_t tb = __float_as_uint(T);
-  const long long e = (long long)((tb >> 23) & 0xFFu) - 127 - 24 + 1023;   // exponent of h+ = ulp(T)/2
-  const double hp = __longlong_as_double(e << 52);
-  const double hm = (tb & 0x7FFFFFu) == 0u ? 0.5 * hp : hp;    // below a power of two the spacing halves
-  const double da = (double)a, db = (double)b, dt = (double)T;
-  if (da > __dmul_rn(dt + hp, db)) return 1;
-  if (da < __dmul_rn(dt - hm, db)) return -1;
+  const float hp = __uint_as_float((tb & 0x7F800000u) - (24u << 23));     // 2^(e_T - 24)
+  const float hm = (tb & 0x7FFFFFu) == 0u ? __fmul_rn(hp, 0.5f) : hp;    // below a power of two the spacing halves
+  const float D = __fmaf_rn(-T, b, a);
+  if (D > __fmul_rn(hp, b)) return 1;
+  if (D < -__fmul_rn(hm, b)) return -1;
   return 0;
+}
+
+// The E2M1 rounding boundary between magnitudes m and m + 1 (m = 0..6):
+// 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.  Their fp32 patterns have zero low 21
+// bits; shifted right by 21 they are 0x1F4 plus 0, 6, 9, 11, 13, 15, 17.
+__device__ __forceinline__ float e2m1_boundary(uint32_t m) {
+  constexpr unsigned long long kOff =
+      (6ull << 5) | (9ull << 10) | (11ull << 15) | (13ull << 20) | (15ull << 25) | (17ull << 30);
+  return __uint_as_float((0x1F4u + (uint32_t)((kOff >> (5u * m)) & 31u)) << 21);
 }
 
 // E2M1 codes of eight values under the two bracketing multipliers: the code
@@ -217,7 +228,7 @@ __device__ __forceinline__ uint2 settle_codes(const T *src, uint64_t lo, uint64_
     const uint32_t cl = (uint32_t)(lo >> sh) & 7u, ch = (uint32_t)(hi >> sh) & 7u;
     const uint32_t mlow = min(cl, ch);
     const float xv = to_f32(src[sh >> 2]);
-    const int c = quotient_vs(fabsf(xv), d, kE2m1Boundary[mlow]);
+    const int c = quotient_vs(fabsf(xv), d, e2m1_boundary(mlow));
     const uint32_t mag = c > 0 ? mlow + 1u : (c < 0 ? mlow : ((mlow & 1u) ? mlow + 1u : mlow));
     const uint32_t code = mag | ((__float_as_uint(xv) >> 28) & 8u);
     lo = (lo & ~(0xFull << sh)) | ((uint64_t)code << sh);

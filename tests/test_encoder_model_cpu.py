@@ -5,8 +5,8 @@ The quantize kernels never divide.  Per block they take
   r = fl32(fl32(1/dec(s)) * fl32(1/g)),  r- = fl32(r (1 - 2^-21)),  r+ = fl32(r (1 + 2^-21)),
 convert fl32(x r-) and fl32(x r+) to E2M1 with round-to-nearest-even and
 saturation, and where the two codes differ they settle the element by
-comparing |x| with (T +- half an ulp of T) * d in fp64, T the E2M1 boundary
-between the two codes, d = fl32(dec(s) g).  The scale byte is chosen the same
+comparing D = fma(-T, d, |x|) (exact near T) with +-half an ulp of T times d,
+T the E2M1 boundary between the two codes, d = fl32(dec(s) g).  The scale byte is chosen the same
 way from amax * fl32(1/fl32(6 g)) widened both ways, settled against the
 midpoint of its two E4M3 candidates.
 
@@ -47,15 +47,27 @@ def e4m3_code(t):
     return np.where(tie & (c % 2 == 1), c + 1, c)
 
 
+def fma32(x, y, z):
+    """fl32(x * y + z) for fp32 x (at most 5 significant bits), y and z: the
+    product is exact in fp64 and so is the sum whenever the exponents of the
+    two terms are within 24 of each other (the only case the rule below needs
+    exactly); farther apart the fp64 sum rounds only bits far below the fp32
+    result."""
+    return (np.asarray(x, np.float64) * np.asarray(y, np.float64) + np.asarray(z, np.float64)).astype(np.float32)
+
+
 def settle(a, b, T):
-    """Sign of fl32(a / b) - T, decided exactly in fp64 (the kernels' rule):
-    above T + h+ rounds above T, below T - h- rounds below, in between is T."""
+    """Sign of fl32(a / b) - T as the kernels decide it: D = fma(-T, b, a) in
+    fp32, then above h+ * b rounds above T, below -h- * b rounds below, in
+    between is T (h+- half the float spacing above and below T)."""
     T = np.asarray(T, np.float32)
     bits = T.view(np.uint32).astype(np.int64)
-    hp = np.ldexp(1.0, ((bits >> 23) & 0xFF) - 127 - 24)                       # half an ulp above T
-    hm = np.where((bits & 0x7FFFFF) == 0, hp / 2, hp)                            # below a power of two
-    a64, b64, t64 = a.astype(np.float64), b.astype(np.float64), T.astype(np.float64)
-    return np.where(a64 > (t64 + hp) * b64, 1, np.where(a64 < (t64 - hm) * b64, -1, 0))
+    hp = np.ldexp(np.float32(1.0), (((bits >> 23) & 0xFF) - 127 - 24).astype(np.int32)).astype(np.float32)
+    hm = np.where((bits & 0x7FFFFF) == 0, hp / F32(2), hp).astype(np.float32)
+    D = fma32(-T, np.asarray(b, np.float32), np.asarray(a, np.float32))
+    up = (hp * np.asarray(b, np.float32)).astype(np.float32)
+    dn = (hm * np.asarray(b, np.float32)).astype(np.float32)
+    return np.where(D > up, 1, np.where(D < -dn, -1, 0))
 
 
 def pick(lo, hi, c):
