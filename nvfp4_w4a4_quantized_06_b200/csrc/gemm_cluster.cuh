@@ -74,10 +74,24 @@ struct ClusterCfg {
   static constexpr int TMEM_COLS = TMEM_NEEDED <= 64 ? 64 : TMEM_NEEDED <= 128 ? 128
                                   : TMEM_NEEDED <= 256 ? 256 : 512;
   static constexpr int MAX_SPLITS = 8;
-  // reduction slots: S slots, each one owner's share of ceil(128/S) tile rows
-  // of RED_PITCH floats (16-byte rows for vector stores); S*ceil(128/S) <= 135
+  // reduction slots: one per rank, each one owner's share of the tile.  A
+  // share is a multiple of 4 tile rows (share_rows), so that the reduction
+  // reads and writes four outputs at a time.  Tile rows i run along the
+  // output's unit stride for decode (the weight is the 128-row operand):
+  // there a slot is [BN columns j][share_rows], otherwise [share rows][BN + 4].
   static constexpr int RED_PITCH = BN + 4;
-  static constexpr int RED_FLOATS = ((BM + MAX_SPLITS - 1) * RED_PITCH + 31) / 32 * 32;   // 128-byte multiple
+  static constexpr int share_rows(int S) { return ((BM + S - 1) / S + 3) / 4 * 4; }
+  static constexpr int slot_floats(int S, bool i_fast) { return i_fast ? BN * share_rows(S) : share_rows(S) * RED_PITCH; }
+  static constexpr int red_need() {
+    int m = 0;
+    for (int S = 1; S <= MAX_SPLITS; ++S) {
+      const int a = S * slot_floats(S, true), b = S * slot_floats(S, false);
+      m = a > m ? a : m;
+      m = b > m ? b : m;
+    }
+    return m;
+  }
+  static constexpr int RED_FLOATS = (red_need() + 31) / 32 * 32;   // 128-byte multiple
   static constexpr int BAR_BYTES = 512;            // barriers, TMEM address, abort flag
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RED_FLOATS * 4 + BAR_BYTES + (FUSED ? 512 : 0);
   static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier area");
@@ -131,6 +145,37 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
   // so a CTA owns whole columns j; otherwise whole rows i
   const bool i_fast = p.out_si == 1;
 
+  // producer helpers (thread 0): the bytes a stage brings and its loads
+  const int row_a = ta * C::BM, row_b = tb * BN;
+  const int pad_b = (p.rows_b + 127) & ~127;
+  const bool a_first = p.group != 0;
+  auto stage_bytes = [&](int ks) {
+    const int nkb = min(4, p.kblocks - ks * 4);
+    int nsfb = 0;
+#pragma unroll
+    for (int j = 0; j < C::SFB_ATOMS; ++j)
+      if (row_b + 128 * j < pad_b) ++nsfb;
+    if (FUSED) return (uint32_t)C::A_BYTES + (uint32_t)nkb * 512u;
+    return (uint32_t)(C::A_BYTES + C::B_BYTES) + (uint32_t)nkb * 512u * (1u + nsfb);
+  };
+  auto load_a = [&](int st, int ks) {
+    const int nkb = min(4, p.kblocks - ks * 4);
+    tma_load_2d(sA + st * C::A_BYTES, &tma, &full[st], ks * 128, row_a);
+    bulk_load(sSFA + st * C::SFA_BYTES, p.sfa + ((int64_t)(row_a >> 7) * p.kblocks + ks * 4) * 512,
+              nkb * 512u, &full[st]);
+  };
+  auto load_b = [&](int st, int ks) {
+    if (FUSED) return;
+    const int nkb = min(4, p.kblocks - ks * 4);
+    tma_load_2d(sB + st * C::B_BYTES, &tmb, &full[st], ks * 128, row_b);
+#pragma unroll
+    for (int j = 0; j < C::SFB_ATOMS; ++j)
+      if (row_b + 128 * j < pad_b)
+        bulk_load(sSFB + st * C::SFB_BYTES + j * 2048,
+                  p.sfb + ((int64_t)((row_b >> 7) + j) * p.kblocks + ks * 4) * 512, nkb * 512u, &full[st]);
+  };
+  const int pre = min(ks1 - ks0, C::STAGES);
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -142,8 +187,13 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
     mbar_init(tdone, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tma);
-    prefetch_tmap(&tmb);
+    // the first ring's worth of the operand that does not depend on the
+    // preceding kernel streams in from here on, while the rest of the CTA
+    // sets up (TMEM, tables) and before the preceding kernel has finished
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&full[i], stage_bytes(ks0 + i));
+      if (a_first) load_a(i, ks0 + i); else load_b(i, ks0 + i);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -166,41 +216,8 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      const int row_a = ta * C::BM, row_b = tb * BN;
-      const int pad_b = (p.rows_b + 127) & ~127;
-      const bool a_first = p.group != 0;
-      auto stage_bytes = [&](int ks) {
-        const int nkb = min(4, p.kblocks - ks * 4);
-        int nsfb = 0;
-#pragma unroll
-        for (int j = 0; j < C::SFB_ATOMS; ++j)
-          if (row_b + 128 * j < pad_b) ++nsfb;
-        if (FUSED) return (uint32_t)C::A_BYTES + (uint32_t)nkb * 512u;
-        return (uint32_t)(C::A_BYTES + C::B_BYTES) + (uint32_t)nkb * 512u * (1u + nsfb);
-      };
-      auto load_a = [&](int st, int ks) {
-        const int nkb = min(4, p.kblocks - ks * 4);
-        tma_load_2d(sA + st * C::A_BYTES, &tma, &full[st], ks * 128, row_a);
-        bulk_load(sSFA + st * C::SFA_BYTES, p.sfa + ((int64_t)(row_a >> 7) * p.kblocks + ks * 4) * 512,
-                  nkb * 512u, &full[st]);
-      };
-      auto load_b = [&](int st, int ks) {
-        if (FUSED) return;
-        const int nkb = min(4, p.kblocks - ks * 4);
-        tma_load_2d(sB + st * C::B_BYTES, &tmb, &full[st], ks * 128, row_b);
-#pragma unroll
-        for (int j = 0; j < C::SFB_ATOMS; ++j)
-          if (row_b + 128 * j < pad_b)
-            bulk_load(sSFB + st * C::SFB_BYTES + j * 2048,
-                      p.sfb + ((int64_t)((row_b >> 7) + j) * p.kblocks + ks * 4) * 512, nkb * 512u, &full[st]);
-      };
-      // the first ring's worth of stages: independent operand first, then
-      // wait for the preceding kernel, then the dependent operand
-      const int pre = min(ks1 - ks0, C::STAGES);
-      for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&full[i], stage_bytes(ks0 + i));
-        if (a_first) load_a(i, ks0 + i); else load_b(i, ks0 + i);
-      }
+      // the independent operand's first stages are in flight (issued at the
+      // top); wait for the preceding kernel, then the dependent operand
       griddep_wait();
       for (int i = 0; i < pre; ++i) {
         if (a_first) load_b(i, ks0 + i); else load_a(i, ks0 + i);
@@ -343,15 +360,16 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
       }
     }
     // ------------------------------- epilogue: partial tile -> owners' slots
-    // Tile row i belongs to rank i*S/128, whose share starts at ceil(r*128/S);
-    // slots are one share (ceil(128/S) rows) apart.
+    // Tile row i belongs to rank i / share; every element goes straight into
+    // the owner's slot named after this rank (distributed-shared-memory
+    // stores).  Decode slots are column-major, so for each column a warp's 32
+    // lanes store 32 consecutive floats.
     const bool ok = mbar_wait_warp(tfull, 0, p.err, ERR_EPILOGUE, abort_flag);
     if (ok) tc_fence_after();
-    const uint32_t slot = (uint32_t)((C::BM + S - 1) / S * C::RED_PITCH);
-    const int own_r = i * S / C::BM;
-    const int row0_r = (own_r * C::BM + S - 1) / S;
-    const uint32_t dst = mapa_shared(smem_u32(red) + (rank * slot + (uint32_t)((i - row0_r) * C::RED_PITCH)) * 4u,
-                                     (uint32_t)own_r);
+    const int share = C::share_rows(S);
+    const int own_r = i / share, a = i - own_r * share;
+    const uint32_t red_rank = mapa_shared(smem_u32(red) + (uint32_t)(rank * C::slot_floats(S, i_fast)) * 4u,
+                                          (uint32_t)own_r);
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t acc[32];
@@ -362,48 +380,87 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
 #pragma unroll
         for (int e = 0; e < 32; ++e) acc[e] = 0u;
       }
+      if (i_fast) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) st_shared_cluster_v4(dst + 4u * (c + e), acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+        for (int e = 0; e < 32; ++e)
+          st_shared_cluster_f32(red_rank + (uint32_t)(((c + e) * share + a) * 4), __uint_as_float(acc[e]));
+      } else {
+        const uint32_t dst = red_rank + (uint32_t)((a * C::RED_PITCH + c) * 4);
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) st_shared_cluster_v4(dst + 4u * e, acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+      }
     }
   }
 
   // ------------------------------------------------- cluster-wide reduction
   // After the barrier every slot of this CTA's share holds the partial of
-  // the rank it is named after; sum them in rank order.  Lanes run along the
-  // output's unit-stride index: the tile row for decode, the column otherwise.
+  // the rank it is named after; sum them in rank order (the result does not
+  // depend on timing).  Each thread takes four outputs that are adjacent
+  // along the output's unit stride: four tile rows of one column for decode,
+  // four columns of one tile row otherwise.
   __syncwarp();                   // reconverge the role warps (the cluster barrier is warp-aligned)
   tc_fence_before();
   cluster_sync();
   {
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
-    const int first = (rank * C::BM + S - 1) / S;
-    const int n_rows = ((rank + 1) * C::BM + S - 1) / S - first;
-    const int slot = (C::BM + S - 1) / S * C::RED_PITCH;
-    // warps step over one index, lanes over the output's unit-stride one
-    const int nw = C::THREADS / 32;
-    const int outer_n = i_fast ? BN : n_rows, inner_n = i_fast ? n_rows : BN;
-    for (int o1 = warp; o1 < outer_n; o1 += nw) {
-      for (int o2 = lane; o2 < inner_n; o2 += 32) {
-        const int a = i_fast ? o2 : o1;                      // row within the share
-        const int j = i_fast ? o1 : o2;
-        const int gi = ta * C::BM + first + a, gj = tb * BN + j;
-        if (gi >= p.rows_a || gj >= p.rows_b) continue;
-        const int off = a * C::RED_PITCH + j;
-        float acc = red[off];
+    const int share = C::share_rows(S);
+    const int first = rank * share;
+    const int n_rows = min(share, C::BM - first);
+    const int slot = C::slot_floats(S, i_fast);
+    // quads: (column, 4 rows) for decode, (row, 4 columns) otherwise
+    const int n_quads = n_rows * BN / 4;
+    const uint32_t red_s = smem_u32(red);
+    for (int t = threadIdx.x; t < n_quads; t += C::THREADS) {
+      int a0, j0, off;
+      if (i_fast) {
+        j0 = t / (n_rows / 4);
+        a0 = (t - j0 * (n_rows / 4)) * 4;
+        off = j0 * share + a0;
+      } else {
+        a0 = t / (BN / 4);
+        j0 = (t - a0 * (BN / 4)) * 4;
+        off = a0 * C::RED_PITCH + j0;
+      }
+      float4 v = ld_shared_f32x4(red_s + (uint32_t)off * 4u);
 #pragma unroll
-        for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
-          if (s2 < S) acc = acc + red[s2 * slot + off];
-        const float v = __fmul_rn(acc, alpha);
-        const int64_t o = (int64_t)gi * p.out_si + (int64_t)gj * p.out_sj;
-        if constexpr (MODE == OUT_BF16) {
-          static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(v);
-        } else if constexpr (MODE == OUT_GATES) {
-          // output column n is the weight row: tile row i for decode-shaped
-          // products, tile column j otherwise
-          const int n = i_fast ? gi : gj;
-          static_cast<float *>(p.out)[o] = n < p.n_split ? gate_keep(v) : gate_write(v);
+      for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
+        if (s2 < S) {
+          const float4 w = ld_shared_f32x4(red_s + (uint32_t)(s2 * slot + off) * 4u);
+          v.x = v.x + w.x; v.y = v.y + w.y; v.z = v.z + w.z; v.w = v.w + w.w;
+        }
+      float o4[4] = {__fmul_rn(v.x, alpha), __fmul_rn(v.y, alpha), __fmul_rn(v.z, alpha), __fmul_rn(v.w, alpha)};
+      const int gi0 = ta * C::BM + first + a0, gj0 = tb * BN + j0;
+      // element q of the quad: (gi0 + q, gj0) for decode, (gi0, gj0 + q) otherwise
+      const int lim = i_fast ? p.rows_a - gi0 : p.rows_b - gj0;
+      if ((i_fast ? gj0 >= p.rows_b : gi0 >= p.rows_a) || lim <= 0) continue;
+      if constexpr (MODE == OUT_GATES) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int n = i_fast ? gi0 + q : gj0 + q;          // output column = weight row
+          o4[q] = n < p.n_split ? gate_keep(o4[q]) : gate_write(o4[q]);
+        }
+      }
+      const int64_t o = (int64_t)gi0 * p.out_si + (int64_t)gj0 * p.out_sj;    // the quad's unit stride is 1
+      if constexpr (MODE == OUT_BF16) {
+        __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.out) + o;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(o4[0], o4[1]), h1 = __floats2bfloat162_rn(o4[2], o4[3]);
+        if (lim >= 4 && (o & 3) == 0) {
+          *reinterpret_cast<uint2 *>(y) =
+              make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
         } else {
-          static_cast<float *>(p.out)[o] = v;
+          const __nv_bfloat16 hv[4] = {h0.x, h0.y, h1.x, h1.y};
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < lim) y[q] = hv[q];
+        }
+      } else {
+        float *y = static_cast<float *>(p.out) + o;
+        if (lim >= 4 && (o & 3) == 0) {
+          *reinterpret_cast<float4 *>(y) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < lim) y[q] = o4[q];
         }
       }
     }

@@ -373,6 +373,13 @@ __device__ __forceinline__ void st_shared_cluster_v4(uint32_t cluster_addr, uint
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+// four floats from this CTA's shared memory (16-byte aligned address)
+__device__ __forceinline__ float4 ld_shared_f32x4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a)
+               : "memory");
+  return v;
+}
 // read a float from the shared memory of a CTA of this cluster
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
   float v;
