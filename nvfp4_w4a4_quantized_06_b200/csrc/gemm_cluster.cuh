@@ -73,22 +73,22 @@ struct ClusterCfg {
   static constexpr int TMEM_NEEDED = BN + STAGES * SF_COLS;
   static constexpr int TMEM_COLS = TMEM_NEEDED <= 64 ? 64 : TMEM_NEEDED <= 128 ? 128
                                   : TMEM_NEEDED <= 256 ? 256 : 512;
-  static constexpr int MAX_SPLITS = 8;
-  // reduction slots: one per rank, each one owner's share of the tile.  A
-  // share is a multiple of 4 tile rows (share_rows), so that the reduction
-  // reads and writes four outputs at a time.  Tile rows i run along the
-  // output's unit stride for decode (the weight is the 128-row operand):
-  // there a slot is [BN columns j][share_rows], otherwise [share rows][BN + 4].
-  static constexpr int RED_PITCH = BN + 4;
+  // cluster sizes this configuration serves (the reduction slots of more
+  // ranks would not fit next to the 128-wide operand ring)
+  static constexpr int MAX_SPLITS = BN >= 128 ? 5 : 8;
+  // reduction slots: one per rank in every owner, holding the owner's share
+  // of the tile, a multiple of 4 tile rows (share_rows).  A slot is
+  // column-major, [BN columns j][slot_pitch], so that for each column the 32
+  // lanes of a warp (32 consecutive tile rows) store 32 consecutive floats,
+  // and the reduction reads four tile rows with one 16-byte load.  The pitch
+  // is the share, plus 4 floats where the share is a multiple of 8, so that
+  // lanes walking over columns hit distinct 16-byte bank groups.
   static constexpr int share_rows(int S) { return ((BM + S - 1) / S + 3) / 4 * 4; }
-  static constexpr int slot_floats(int S, bool i_fast) { return i_fast ? BN * share_rows(S) : share_rows(S) * RED_PITCH; }
+  static constexpr int slot_pitch(int S) { return share_rows(S) % 8 == 0 ? share_rows(S) + 4 : share_rows(S); }
+  static constexpr int slot_floats(int S) { return BN * slot_pitch(S); }
   static constexpr int red_need() {
     int m = 0;
-    for (int S = 1; S <= MAX_SPLITS; ++S) {
-      const int a = S * slot_floats(S, true), b = S * slot_floats(S, false);
-      m = a > m ? a : m;
-      m = b > m ? b : m;
-    }
+    for (int S = 1; S <= MAX_SPLITS; ++S) m = S * slot_floats(S) > m ? S * slot_floats(S) : m;
     return m;
   }
   static constexpr int RED_FLOATS = (red_need() + 31) / 32 * 32;   // 128-byte multiple
@@ -362,16 +362,18 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
     // ------------------------------- epilogue: partial tile -> owners' slots
     // Tile row i belongs to rank i / share; every element goes straight into
     // the owner's slot named after this rank (distributed-shared-memory
-    // stores).  Decode slots are column-major, so for each column a warp's 32
-    // lanes store 32 consecutive floats.
+    // stores; for each column the warp's 32 lanes write 32 consecutive
+    // floats, one transaction).  Columns past the narrow operand's rows hold
+    // zeros and are neither sent nor summed.
     const bool ok = mbar_wait_warp(tfull, 0, p.err, ERR_EPILOGUE, abort_flag);
     if (ok) tc_fence_after();
-    const int share = C::share_rows(S);
+    const int share = C::share_rows(S), pitch = C::slot_pitch(S);
     const int own_r = i / share, a = i - own_r * share;
-    const uint32_t red_rank = mapa_shared(smem_u32(red) + (uint32_t)(rank * C::slot_floats(S, i_fast)) * 4u,
+    const int ncols = min(BN, p.rows_b - tb * BN);
+    const uint32_t red_rank = mapa_shared(smem_u32(red) + (uint32_t)(rank * C::slot_floats(S) + a) * 4u,
                                           (uint32_t)own_r);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = 0; c < ncols; c += 32) {
       uint32_t acc[32];
       if (ok) {
         tmem_ld32(tmem + lane_addr + c, acc);
@@ -380,87 +382,81 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
 #pragma unroll
         for (int e = 0; e < 32; ++e) acc[e] = 0u;
       }
-      if (i_fast) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          st_shared_cluster_f32(red_rank + (uint32_t)(((c + e) * share + a) * 4), __uint_as_float(acc[e]));
-      } else {
-        const uint32_t dst = red_rank + (uint32_t)((a * C::RED_PITCH + c) * 4);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) st_shared_cluster_v4(dst + 4u * e, acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
-      }
+      for (int e = 0; e < 32; ++e)
+        st_shared_cluster_f32(red_rank + (uint32_t)((c + e) * pitch * 4), __uint_as_float(acc[e]));
     }
   }
 
   // ------------------------------------------------- cluster-wide reduction
   // After the barrier every slot of this CTA's share holds the partial of
   // the rank it is named after; sum them in rank order (the result does not
-  // depend on timing).  Each thread takes four outputs that are adjacent
-  // along the output's unit stride: four tile rows of one column for decode,
-  // four columns of one tile row otherwise.
+  // depend on timing).  Each thread takes four consecutive tile rows of one
+  // column (one 16-byte load per slot).  For decode the tile rows run along
+  // the output's unit stride: lanes walk over row quads and each writes its
+  // four outputs at once.  Otherwise lanes walk over columns, the output's
+  // unit stride, and write one row at a time.
   __syncwarp();                   // reconverge the role warps (the cluster barrier is warp-aligned)
   tc_fence_before();
   cluster_sync();
   {
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
-    const int share = C::share_rows(S);
+    const int share = C::share_rows(S), pitch = C::slot_pitch(S);
     const int first = rank * share;
-    const int n_rows = min(share, C::BM - first);
-    const int slot = C::slot_floats(S, i_fast);
-    // quads: (column, 4 rows) for decode, (row, 4 columns) otherwise
-    const int n_quads = n_rows * BN / 4;
+    const int n_quads = min(share, C::BM - first) / 4;
+    const int ncols = min(BN, p.rows_b - tb * BN);
+    const int slot = C::slot_floats(S);
     const uint32_t red_s = smem_u32(red);
-    for (int t = threadIdx.x; t < n_quads; t += C::THREADS) {
-      int a0, j0, off;
+    for (int t = threadIdx.x; t < n_quads * ncols; t += C::THREADS) {
+      int j, aq;
       if (i_fast) {
-        j0 = t / (n_rows / 4);
-        a0 = (t - j0 * (n_rows / 4)) * 4;
-        off = j0 * share + a0;
+        j = t / n_quads;
+        aq = t - j * n_quads;
       } else {
-        a0 = t / (BN / 4);
-        j0 = (t - a0 * (BN / 4)) * 4;
-        off = a0 * C::RED_PITCH + j0;
+        aq = t / ncols;
+        j = t - aq * ncols;
       }
-      float4 v = ld_shared_f32x4(red_s + (uint32_t)off * 4u);
+      const int a0 = aq * 4;
+      const uint32_t off = (uint32_t)(j * pitch + a0) * 4u;
+      float4 v = ld_shared_f32x4(red_s + off);
 #pragma unroll
       for (int s2 = 1; s2 < C::MAX_SPLITS; ++s2)
         if (s2 < S) {
-          const float4 w = ld_shared_f32x4(red_s + (uint32_t)(s2 * slot + off) * 4u);
+          const float4 w = ld_shared_f32x4(red_s + off + (uint32_t)(s2 * slot) * 4u);
           v.x = v.x + w.x; v.y = v.y + w.y; v.z = v.z + w.z; v.w = v.w + w.w;
         }
       float o4[4] = {__fmul_rn(v.x, alpha), __fmul_rn(v.y, alpha), __fmul_rn(v.z, alpha), __fmul_rn(v.w, alpha)};
-      const int gi0 = ta * C::BM + first + a0, gj0 = tb * BN + j0;
-      // element q of the quad: (gi0 + q, gj0) for decode, (gi0, gj0 + q) otherwise
-      const int lim = i_fast ? p.rows_a - gi0 : p.rows_b - gj0;
-      if ((i_fast ? gj0 >= p.rows_b : gi0 >= p.rows_a) || lim <= 0) continue;
+      const int gi0 = ta * C::BM + first + a0, gj = tb * BN + j;
+      const int lim = p.rows_a - gi0;              // valid tile rows of the quad
+      if (lim <= 0) continue;
       if constexpr (MODE == OUT_GATES) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int n = i_fast ? gi0 + q : gj0 + q;          // output column = weight row
+          const int n = i_fast ? gi0 + q : gj;             // output column = weight row
           o4[q] = n < p.n_split ? gate_keep(o4[q]) : gate_write(o4[q]);
         }
       }
-      const int64_t o = (int64_t)gi0 * p.out_si + (int64_t)gj0 * p.out_sj;    // the quad's unit stride is 1
+      const int64_t o = (int64_t)gi0 * p.out_si + (int64_t)gj * p.out_sj;
       if constexpr (MODE == OUT_BF16) {
         __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.out) + o;
         __nv_bfloat162 h0 = __floats2bfloat162_rn(o4[0], o4[1]), h1 = __floats2bfloat162_rn(o4[2], o4[3]);
-        if (lim >= 4 && (o & 3) == 0) {
+        if (i_fast && lim >= 4 && (o & 3) == 0) {
           *reinterpret_cast<uint2 *>(y) =
               make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
         } else {
           const __nv_bfloat16 hv[4] = {h0.x, h0.y, h1.x, h1.y};
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            if (q < lim) y[q] = hv[q];
+            if (q < lim) y[(int64_t)q * p.out_si] = hv[q];
         }
       } else {
         float *y = static_cast<float *>(p.out) + o;
-        if (lim >= 4 && (o & 3) == 0) {
+        if (i_fast && lim >= 4 && (o & 3) == 0) {
           *reinterpret_cast<float4 *>(y) = make_float4(o4[0], o4[1], o4[2], o4[3]);
         } else {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            if (q < lim) y[q] = o4[q];
+            if (q < lim) y[(int64_t)q * p.out_si] = o4[q];
         }
       }
     }

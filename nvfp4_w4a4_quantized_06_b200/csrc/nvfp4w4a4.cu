@@ -150,6 +150,9 @@ nvfp4_status device_state(DeviceState **out) {
         set_cluster_attrs<64>() != cudaSuccess || set_cluster_attrs<128>() != cudaSuccess ||
         set_quant_attrs<__nv_bfloat16>() != cudaSuccess || set_quant_attrs<float>() != cudaSuccess)
       return NVFP4_ERR_CUDA;
+    static_assert(ClusterCfg<32>::MAX_SPLITS == kMaxSplitCluster && ClusterCfg<64>::MAX_SPLITS == kMaxSplitCluster &&
+                      ClusterCfg<128>::MAX_SPLITS == 5,
+                  "planner limits follow the reduction slots");
     for (int c = 1; c <= kMaxSplitCluster; ++c) {
       d.split_clusters[0][c] = max_split_clusters<32>(c, sms);
       d.split_clusters[1][c] = max_split_clusters<64>(c, sms);
@@ -236,6 +239,8 @@ struct Plan {
 };
 
 inline int narrow_bn(int64_t rows) { return rows <= 32 ? 32 : (rows <= 64 ? 64 : 128); }
+// largest split-K cluster a configuration's reduction slots hold (ClusterCfg::MAX_SPLITS)
+inline int max_splits_for_bn(int bn) { return bn >= 128 ? 5 : kMaxSplitCluster; }
 inline int bn_index(int bn) { return bn == 32 ? 0 : (bn == 64 ? 1 : 2); }
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, const DeviceState &d) {
@@ -266,7 +271,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, const DeviceState &d) {
     pl.tiles_b = 1;
     int best = 0;
     int64_t best_cost = 0;
-    for (int c = 1; c <= kMaxSplitCluster && c <= pl.kstages; ++c) {
+    for (int c = 1; c <= max_splits_for_bn(pl.bn) && c <= pl.kstages; ++c) {
       const int fit = d.split_clusters[bn_index(pl.bn)][c];
       if (fit <= 0) continue;
       const int64_t waves = (pl.tiles_a + fit - 1) / fit;

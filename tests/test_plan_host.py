@@ -20,10 +20,11 @@ def _lib():
     native.lib()
 
 
-def best_split(tiles, kstages, fit):
-    """Cluster size minimising waves x (stages per CTA + 1), first on ties."""
+def best_split(tiles, kstages, fit, bn=32):
+    """Cluster size minimising waves x (stages per CTA + 1), first on ties;
+    a 128-wide MMA N allows clusters of up to 5 CTAs (its reduction slots)."""
     best, cost = 0, None
-    for c in range(1, min(8, kstages) + 1):
+    for c in range(1, min(5 if bn >= 128 else 8, kstages) + 1):
         if fit[c] <= 0:
             continue
         k = math.ceil(tiles / fit[c]) * (math.ceil(kstages / c) + 1)
@@ -50,7 +51,7 @@ def test_every_configuration_gets_its_kernel():
             assert p["bn"] == (32 if narrow <= 32 else 64 if narrow <= 64 else 128)
             tiles = math.ceil((N if swap else M) / 128)
             assert p["tiles_a"] == tiles
-            assert p["splits"] == best_split(tiles, p["kstages"], SPLITS[0])
+            assert p["splits"] == best_split(tiles, p["kstages"], SPLITS[0], p["bn"])
             assert p["grid"] == tiles * p["splits"]
 
 
