@@ -177,6 +177,9 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
   const int pre = min(ks1 - ks0, C::STAGES);
 
   if (threadIdx.x == 0) {
+    // the tensor maps' descriptors are fetched while the barriers are set up
+    prefetch_tmap(&tma);
+    if (!FUSED) prefetch_tmap(&tmb);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
