@@ -337,94 +337,20 @@ def measure_e2e(native, x_cpu, gx, w_codes, w_sf, gw, M, N, K, dev, world, steps
             "d2h_bytes_per_step": y_host.numel() * 2}
 
 
-def measure_secondary(native, dev):
-    """The other workloads of the layer, one line each (median of events):
-    GDN fused groups (TFLOP/s), decode shapes (HBM GB/s over weights+X+Y,
-    rotating over >= 4x L2 of weight copies inside a CUDA graph)."""
+SECONDARY = ("gdn_qkv_z", "gdn_gates_ab", "decode_out_proj", "decode_down_proj", "gdn_gates_fused_activations",
+             "fake_quant_bf16", "fp8_kv_quantize", "rmsnorm_quantize", "harmonize_requant_qkv_z")
+
+
+def measure_secondary(native, dev, only=None):
+    """The other workloads of the layer and the rows built beyond it, one line
+    each (median of CUDA events): GDN fused groups (TFLOP/s), decode shapes
+    (HBM GB/s over weights+X+Y, rotating over >= 4x L2 of weight copies inside
+    a CUDA graph), then the gate epilogue, fake-quant, FP8 KV quantize, the
+    RMSNorm-fused quantize and the re-quantizing harmonize.  `only`: a set of
+    line names to run (all when None)."""
     res = {}
     pk = peaks()
-    for name in ("gdn_qkv_z", "gdn_gates_ab"):
-        wl = W.WORKLOADS[name]
-        x = W.make_x(wl).to(dev)
-        wc, wsf, gw = quantized_weight(wl, dev)
-        gx = native.amax_gscale(x)
-        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
-        flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
-        times = []
-        for i in range(12):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            native.linear(x, gx, wc, wsf, gw, out=y, workspace=ws)
-            e1.record()
-            torch.cuda.synchronize()
-            if i >= 2:
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
-        byts = wl.M * wl.K * 2 + wl.N * wl.K // 2 + wl.N * wl.K // 16 + wl.M * wl.N * 2
-        res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4),
-                     "tflops": round(wl.flops / (ms * 1e-3) / 1e12, 1),
-                     "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                     "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
-                     "l2": "512 MB flush between reps"}
-        del x, wc, wsf, y, ws, flush
-    for name in ("decode_out_proj", "decode_down_proj"):
-        wl = W.WORKLOADS[name]
-        x = W.make_x(wl).to(dev)
-        wc, wsf, gw = quantized_weight(wl, dev)
-        gx = native.amax_gscale(x)
-        wbytes = wc.numel() + wsf.numel()
-        copies = max(4, int(np.ceil(4 * 126e6 / wbytes)))
-        wcs = [wc.clone() for _ in range(copies)]
-        wsfs = [wsf.clone() for _ in range(copies)]
-        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
-        for i in range(copies):                   # warm-up outside capture
-            native.linear(x, gx, wcs[i], wsfs[i], gw, out=y, workspace=ws)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(copies):
-                native.linear(x, gx, wcs[i], wsfs[i], gw, out=y, workspace=ws)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 5
-        e0.record()
-        for _ in range(reps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / (reps * copies)
-        byts = wbytes + wl.M * wl.K * 2 + wl.M * wl.N * 2
-        res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "us": round(ms * 1e3, 2),
-                     "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                     "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
-                     "l2": f"CUDA graph over {copies} weight copies ({copies * wbytes / 1e6:.0f} MB)"}
-        # the same calls through the one-kernel variant (activation quantized in the GEMM)
-        gf = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gf):
-            for i in range(copies):
-                native.linear_fused(x, gx, wcs[i], wsfs[i], gw, out=y)
-        gf.replay()
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(reps):
-            gf.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        msf = e0.elapsed_time(e1) / (reps * copies)
-        res[name]["fused_prologue_us"] = round(msf * 1e3, 2)
-        del gf
-        del g, wcs, wsfs, x, y, ws
-    # rows beyond the layer: fused gate epilogue, fake-quant, FP8 KV quantize
-    wl = W.WORKLOADS["gdn_gates_ab"]
-    x = W.make_x(wl).to(dev)
-    wc, wsf, gw = quantized_weight(wl, dev)
-    gx = native.amax_gscale(x)
-    out = torch.empty((wl.M, wl.N), dtype=torch.float32, device=dev)
-    ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+    want = (lambda name: True) if only is None else (lambda name: name in only)
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
 
     def timed(fn, reps=12):
@@ -440,68 +366,133 @@ def measure_secondary(native, dev):
                 times.append(e0.elapsed_time(e1))
         return statistics.median(times)
 
-    ms = timed(lambda: native.gdn_gates(x, gx, wc, wsf, gw, n_a=wl.modules[0], out=out, workspace=ws))
-    byts = wl.M * wl.K * 2 + wl.N * wl.K // 2 + wl.N * wl.K // 16 + wl.M * wl.N * 4
-    res["gdn_gates_fused_activations"] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4),
-                                          "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                                          "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
-                                          "l2": "512 MB flush between reps"}
-    del x, wc, wsf, out, ws
+    def hbm(byts, ms):
+        return {"gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
+                "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3)}
+
+    for name in ("gdn_qkv_z", "gdn_gates_ab"):
+        if not want(name):
+            continue
+        wl = W.WORKLOADS[name]
+        x = W.make_x(wl).to(dev)
+        wc, wsf, gw = quantized_weight(wl, dev)
+        gx = native.amax_gscale(x)
+        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: native.linear(x, gx, wc, wsf, gw, out=y, workspace=ws))
+        byts = wl.M * wl.K * 2 + wl.N * wl.K // 2 + wl.N * wl.K // 16 + wl.M * wl.N * 2
+        res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4),
+                     "tflops": round(wl.flops / (ms * 1e-3) / 1e12, 1), **hbm(byts, ms),
+                     "l2": "512 MB flush between reps"}
+        del x, wc, wsf, y, ws
+    for name in ("decode_out_proj", "decode_down_proj"):
+        if not want(name):
+            continue
+        wl = W.WORKLOADS[name]
+        x = W.make_x(wl).to(dev)
+        wc, wsf, gw = quantized_weight(wl, dev)
+        gx = native.amax_gscale(x)
+        wbytes = wc.numel() + wsf.numel()
+        copies = max(4, int(np.ceil(4 * 126e6 / wbytes)))
+        wcs = [wc.clone() for _ in range(copies)]
+        wsfs = [wsf.clone() for _ in range(copies)]
+        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+        for i in range(copies):                   # warm-up outside capture
+            native.linear(x, gx, wcs[i], wsfs[i], gw, out=y, workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        per_call = {}
+        for label, fn in (("layer", native.linear), ("fused", None)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(copies):
+                    if fn is None:
+                        native.linear_fused(x, gx, wcs[i], wsfs[i], gw, out=y)
+                    else:
+                        fn(x, gx, wcs[i], wsfs[i], gw, out=y, workspace=ws)
+            g.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            per_call[label] = e0.elapsed_time(e1) / (reps * copies)
+            del g
+        ms = per_call["layer"]
+        byts = wbytes + wl.M * wl.K * 2 + wl.M * wl.N * 2
+        res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "us": round(ms * 1e3, 2), **hbm(byts, ms),
+                     "l2": f"CUDA graph over {copies} weight copies ({copies * wbytes / 1e6:.0f} MB)",
+                     # the same calls through the one-kernel variant (activation quantized in the GEMM)
+                     "fused_prologue_us": round(per_call["fused"] * 1e3, 2)}
+        del wcs, wsfs, x, y, ws
+    if want("gdn_gates_fused_activations"):
+        wl = W.WORKLOADS["gdn_gates_ab"]
+        x = W.make_x(wl).to(dev)
+        wc, wsf, gw = quantized_weight(wl, dev)
+        gx = native.amax_gscale(x)
+        out = torch.empty((wl.M, wl.N), dtype=torch.float32, device=dev)
+        ws = torch.empty(native.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: native.gdn_gates(x, gx, wc, wsf, gw, n_a=wl.modules[0], out=out, workspace=ws))
+        byts = wl.M * wl.K * 2 + wl.N * wl.K // 2 + wl.N * wl.K // 16 + wl.M * wl.N * 4
+        res["gdn_gates_fused_activations"] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4), **hbm(byts, ms),
+                                              "l2": "512 MB flush between reps"}
+        del x, wc, wsf, out, ws
     wl = W.WORKLOADS["prefill_mlp_gate_up"]
-    x = W.make_x(wl).to(dev)
-    g = native.amax_gscale(x)
-    fq = torch.empty_like(x)
-    st = torch.empty(2, dtype=torch.float64, device=dev)
-    ms = timed(lambda: native.lib().nvfp4_fake_quant(x.data_ptr(), 0, wl.M, wl.K, wl.K, g.data_ptr(), fq.data_ptr(), 0,
-                                                     wl.K, st.data_ptr(), torch.cuda.current_stream().cuda_stream))
-    byts = wl.M * wl.K * 4
-    res["fake_quant_bf16"] = {"shape": f"{wl.M}x{wl.K}", "ms": round(ms, 4),
-                              "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                              "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
-                              "rel_error": round(float(np.sqrt(st[0].item() / st[1].item())), 5)}
-    del fq
-    kv = torch.randn(32 * 4096 * 4 * 256 * 2, dtype=torch.bfloat16, device=dev)     # 32 seqs x 4096 tokens, K and V
-    sc = (kv.abs().max().float() / 448.0).reshape(1)
-    q8 = torch.empty(kv.numel(), dtype=torch.uint8, device=dev)
-    ms = timed(lambda: native.fp8_quantize(kv, sc, out=q8))
-    byts = kv.numel() * 3
-    res["fp8_kv_quantize"] = {"shape": "32x4096 tokens x 4 kv heads x 256 x (K,V) bf16", "ms": round(ms, 4),
-                              "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                              "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3)}
-    del kv, q8
-    # quantize fused into the RMSNorm that produces this activation
-    wn = W.norm_weight(wl.K, seed=11).to(dev)
-    gy = native.amax_gscale(torch.nn.functional.rms_norm(x, (wl.K,), weight=wn, eps=1e-6))
-    yc = torch.empty((wl.M, wl.K // 2), dtype=torch.uint8, device=dev)
-    ysf = torch.empty(native.sf_bytes(wl.M, wl.K), dtype=torch.uint8, device=dev)
-    yinv = torch.empty(wl.M, dtype=torch.float32, device=dev)
-    ms = timed(lambda: native.rmsnorm_quantize(x, wn, 1e-6, gy, codes=yc, sf=ysf, inv=yinv))
+    x = W.make_x(wl).to(dev) if (want("fake_quant_bf16") or want("rmsnorm_quantize")) else None
+    if want("fake_quant_bf16"):
+        g = native.amax_gscale(x)
+        fq = torch.empty_like(x)
+        st = torch.empty(2, dtype=torch.float64, device=dev)
+        ms = timed(lambda: native.lib().nvfp4_fake_quant(x.data_ptr(), 0, wl.M, wl.K, wl.K, g.data_ptr(), fq.data_ptr(),
+                                                         0, wl.K, st.data_ptr(),
+                                                         torch.cuda.current_stream().cuda_stream))
+        res["fake_quant_bf16"] = {"shape": f"{wl.M}x{wl.K}", "ms": round(ms, 4), **hbm(wl.M * wl.K * 4, ms),
+                                  "rel_error": round(float(np.sqrt(st[0].item() / st[1].item())), 5)}
+        del fq
+    if want("fp8_kv_quantize"):
+        kv = torch.randn(32 * 4096 * 4 * 256 * 2, dtype=torch.bfloat16, device=dev)     # 32 seqs x 4096 tokens, K and V
+        sc = (kv.abs().max().float() / 448.0).reshape(1)
+        q8 = torch.empty(kv.numel(), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: native.fp8_quantize(kv, sc, out=q8))
+        res["fp8_kv_quantize"] = {"shape": "32x4096 tokens x 4 kv heads x 256 x (K,V) bf16", "ms": round(ms, 4),
+                                  **hbm(kv.numel() * 3, ms)}
+        del kv, q8
+    if want("rmsnorm_quantize"):
+        # quantize fused into the RMSNorm that produces this activation
+        wn = W.norm_weight(wl.K, seed=11).to(dev)
+        gy = native.amax_gscale(torch.nn.functional.rms_norm(x, (wl.K,), weight=wn, eps=1e-6))
+        yc = torch.empty((wl.M, wl.K // 2), dtype=torch.uint8, device=dev)
+        ysf = torch.empty(native.sf_bytes(wl.M, wl.K), dtype=torch.uint8, device=dev)
+        yinv = torch.empty(wl.M, dtype=torch.float32, device=dev)
+        ms = timed(lambda: native.rmsnorm_quantize(x, wn, 1e-6, gy, codes=yc, sf=ysf, inv=yinv))
 
-    def unfused():
-        y = torch.nn.functional.rms_norm(x, (wl.K,), weight=wn, eps=1e-6)
-        native.quantize(y, gy, codes=yc, sf=ysf)
+        def unfused():
+            y = torch.nn.functional.rms_norm(x, (wl.K,), weight=wn, eps=1e-6)
+            native.quantize(y, gy, codes=yc, sf=ysf)
 
-    ms_unfused = timed(unfused)
-    byts = wl.M * wl.K * 2 + wl.M * wl.K // 2 + wl.M * wl.K // 16 + wl.K * 2 + wl.M * 4
-    res["rmsnorm_quantize"] = {"shape": f"{wl.M}x{wl.K} bf16 residual", "ms": round(ms, 4),
-                               "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                               "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
-                               "unfused_torch_rms_norm_then_quantize_ms": round(ms_unfused, 4),
-                               "l2": "512 MB flush between reps"}
-    del x, yc, ysf, yinv
-    # re-quantizing harmonize of the fused qkv+z weight (offline; in place, so
-    # every rep re-encodes the previous rep's output)
-    wl = W.WORKLOADS["gdn_qkv_z"]
-    wc, wsf, gw = quantized_weight(wl, dev)
-    offs = [0, wl.modules[0], wl.N]
-    gsm = torch.cat([gw, gw * 0.8])
-    ms = timed(lambda: native.harmonize_requant(wc, wsf, wl.K, offs, gsm))
-    byts = 2 * (wl.N * wl.K // 2 + wl.N * wl.K // 16)
-    res["harmonize_requant_qkv_z"] = {"shape": f"{wl.N}x{wl.K}", "ms": round(ms, 4),
-                                      "gbs_algorithmic": round(byts / (ms * 1e-3) / 1e9, 1),
-                                      "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 3),
-                                      "l2": "512 MB flush between reps"}
-    del wc, wsf, flush
+        ms_unfused = timed(unfused)
+        byts = wl.M * wl.K * 2 + wl.M * wl.K // 2 + wl.M * wl.K // 16 + wl.K * 2 + wl.M * 4
+        res["rmsnorm_quantize"] = {"shape": f"{wl.M}x{wl.K} bf16 residual", "ms": round(ms, 4), **hbm(byts, ms),
+                                   "unfused_torch_rms_norm_then_quantize_ms": round(ms_unfused, 4),
+                                   "l2": "512 MB flush between reps"}
+        del yc, ysf, yinv
+    del x
+    if want("harmonize_requant_qkv_z"):
+        # re-quantizing harmonize of the fused qkv+z weight (offline; in place, so
+        # every rep re-encodes the previous rep's output)
+        wl = W.WORKLOADS["gdn_qkv_z"]
+        wc, wsf, gw = quantized_weight(wl, dev)
+        offs = [0, wl.modules[0], wl.N]
+        gsm = torch.cat([gw, gw * 0.8])
+        ms = timed(lambda: native.harmonize_requant(wc, wsf, wl.K, offs, gsm))
+        byts = 2 * (wl.N * wl.K // 2 + wl.N * wl.K // 16)
+        res["harmonize_requant_qkv_z"] = {"shape": f"{wl.N}x{wl.K}", "ms": round(ms, 4), **hbm(byts, ms),
+                                          "l2": "512 MB flush between reps"}
+        del wc, wsf
+    del flush
     assert native.last_device_status() == 0
     return res
 
@@ -622,6 +613,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--oracle-table", action="store_true",
                     help="time the CPU oracle on every configuration (host cores only) and exit")
+    ap.add_argument("--only", default=None,
+                    help="comma-separated secondary lines to measure instead of the headline "
+                         f"(one GPU; any of {', '.join(SECONDARY)}); prints them as one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -640,6 +634,14 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.only is not None:
+        names = {n.strip() for n in args.only.split(",") if n.strip()}
+        unknown = names - set(SECONDARY)
+        if unknown:
+            raise SystemExit(f"--only: unknown line(s) {sorted(unknown)}; choose from {list(SECONDARY)}")
+        from nvfp4_w4a4_quantized_06_b200 import native
+        print(json.dumps({"only": measure_secondary(native, dev, only=names)}), flush=True)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),

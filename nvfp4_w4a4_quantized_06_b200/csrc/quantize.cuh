@@ -16,6 +16,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -522,6 +523,33 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
   return __uint_as_float(bits | ((c & 8u) << 28));
 }
 
+// Sixteen E2M1 codes (w.x holds elements 0-7, element 2j in the low nibble of
+// byte j) times an E4M3 scale value ds, as floats: the conversion instruction
+// takes one byte (two codes) to two halves, one half-precision multiply by ds
+// (exact: the products have at most 6 significant bits and stay in the normal
+// half range), then the widening to fp32 (exact).
+__device__ __forceinline__ void e2m1x16_times_scale(uint2 w, float ds, float (&out)[16]) {
+  const __half2 s2 = __float2half2_rn(ds);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t p[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3])
+        : "r"(h ? w.y : w.x));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 q = __hmul2(*reinterpret_cast<const __half2 *>(&p[j]), s2);
+      out[8 * h + 2 * j] = __low2float(q);
+      out[8 * h + 2 * j + 1] = __high2float(q);
+    }
+  }
+}
+
 struct FakeQuantParams {
   const void *x;
   int64_t rows, K, ld_x;
@@ -557,7 +585,7 @@ __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16 *dst, const
 // squared input.  One warp per 512-column
 // row segment, lane l owning block l, like quantize_rows_kernel.
 template <typename T, typename OUT>
-__global__ void __launch_bounds__(256) fake_quant_kernel(FakeQuantParams p) {
+__global__ void __launch_bounds__(256, 4) fake_quant_kernel(FakeQuantParams p) {
   __shared__ float rcp_tab[128];
   fill_rcp_table(rcp_tab);
   pdl_prologue();
@@ -593,12 +621,15 @@ __global__ void __launch_bounds__(256) fake_quant_kernel(FakeQuantParams p) {
     const Block16<T> &b = bb[h];
     uint32_t s;
     const uint2 w = encode16(b, kc, rcp_tab, src, &s);
-    const float ds = e4m3_to_f32(s);
+    // dec(q) * dec(s): the hardware turns two codes into two halves, and their
+    // product with the scale is exact in f16 (at most 6 significant bits,
+    // magnitudes from 2^-10 to 2688)
+    float qv[16];
+    e2m1x16_times_scale(w, e4m3_to_f32(s), qv);
     float v[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const uint32_t c = ((e < 8 ? w.x : w.y) >> ((e & 7) * 4)) & 0xFu;
-      const float qs = __fmul_rn(e2m1_to_f32(c), ds);            // exact: at most 7 significant bits
+      const float qs = qv[e];
       v[e] = __fmul_rn(qs, kc.g);
       // the error is taken against the exact NVFP4 value (exact in float64)
       const double xe = (double)b.elem(e), d = xe - (double)qs * (double)kc.g;
@@ -633,18 +664,60 @@ struct Fp8Params {
   uint8_t *q;
 };
 
-__device__ __forceinline__ uint32_t fp8_settle(float x, float s, uint32_t lo, uint32_t hi) {
+// Midpoints between neighbouring E4M3 magnitudes: mid[m] = (dec(m) + dec(m + 1)) / 2
+// for m = 0..125 (exact in fp32: at most five significant bits).
+__device__ __forceinline__ void fill_e4m3_mid_table(float *tab) {
+  for (int i = threadIdx.x; i < 128; i += blockDim.x)
+    tab[i] = i < 126 ? __fmul_rn(__fadd_rn(e4m3_to_f32((uint32_t)i), e4m3_to_f32((uint32_t)i + 1u)), 0.5f) : 0.0f;
+}
+
+// The code of x where the two bracketing conversions disagree (neighbouring
+// magnitudes m0 < m1): above their midpoint m1, below m0, on it the even one.
+__device__ __forceinline__ uint32_t fp8_settle(float x, float s, uint32_t lo, uint32_t hi, const float *mid_tab) {
   const uint32_t ml = lo & 0x7Fu, mh = hi & 0x7Fu;
   const uint32_t m0 = min(ml, mh), m1 = max(ml, mh);
-  const float mid = __fmul_rn(__fadd_rn(e4m3_to_f32(m0), e4m3_to_f32(m1)), 0.5f);
-  const int c = quotient_vs(fabsf(x), s, mid);
+  const int c = quotient_vs(fabsf(x), s, mid_tab[m0]);
   const uint32_t m = c > 0 ? m1 : (c < 0 ? m0 : ((m0 & 1u) ? m1 : m0));
   return m | (__float_as_uint(x) >> 24 & 0x80u);
 }
 
+// Eight values to eight E4M3 codes (byte j = element j).  Each conversion
+// instruction takes two elements; the words from the two bracketing
+// multipliers are compared whole, and only bytes that differ are settled.
+__device__ __forceinline__ uint2 fp8x8(const float (&v)[8], float s, float rlo, float rhi, const float *mid_tab) {
+  uint32_t lo[2], hi[2];
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    uint16_t l0, l1, h0, h1;
+    const float *e = v + 4 * w;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(l0) : "f"(__fmul_rn(e[1], rlo)), "f"(__fmul_rn(e[0], rlo)));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(l1) : "f"(__fmul_rn(e[3], rlo)), "f"(__fmul_rn(e[2], rlo)));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h0) : "f"(__fmul_rn(e[1], rhi)), "f"(__fmul_rn(e[0], rhi)));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h1) : "f"(__fmul_rn(e[3], rhi)), "f"(__fmul_rn(e[2], rhi)));
+    lo[w] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+    hi[w] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+  }
+  const uint32_t d0 = lo[0] ^ hi[0], d1 = lo[1] ^ hi[1];
+  if ((d0 | d1) != 0u) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t dk = (k < 4 ? d0 : d1) >> ((k & 3) * 8) & 0xFFu;
+      if (dk != 0u) {
+        const int w = k >> 2, sh = (k & 3) * 8;
+        const uint32_t code = fp8_settle(v[k], s, lo[w] >> sh & 0xFFu, hi[w] >> sh & 0xFFu, mid_tab);
+        lo[w] = (lo[w] & ~(0xFFu << sh)) | (code << sh);
+      }
+    }
+  }
+  return make_uint2(lo[0], lo[1]);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) fp8_quantize_kernel(Fp8Params p) {
+  __shared__ float mid_tab[128];
+  fill_e4m3_mid_table(mid_tab);
   pdl_prologue();
+  __syncthreads();
   const float s = __ldg(p.scale);
   const bool fast = s >= 8.67361738e-19f && s <= 1.15292150e18f;   // 2^-60 .. 2^60
   const float rs = __frcp_rn(s);
@@ -683,23 +756,20 @@ __global__ void __launch_bounds__(256) fp8_quantize_kernel(Fp8Params p) {
     for (int c = 0; c < U; ++c) {
       const int64_t i = base + c * nthreads;
       if (i >= chunks) continue;
-      uint32_t out[2] = {0u, 0u};
+      uint2 out;
+      if (fast) {
+        out = fp8x8(v[c], s, rlo, rhi, mid_tab);
+      } else {
+        uint32_t o[2] = {0u, 0u};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        uint32_t code;
-        if (fast) {
-          uint16_t pr;
-          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(__fmul_rn(v[c][k], rhi)), "f"(__fmul_rn(v[c][k], rlo)));
-          const uint32_t lo = pr & 0xFFu, hi = (uint32_t)(pr >> 8);
-          code = lo == hi ? lo : fp8_settle(v[c][k], s, lo, hi);
-        } else {
+        for (int k = 0; k < 8; ++k) {
           uint16_t pr;
           asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(0.0f), "f"(div_rn_slow(v[c][k], s)));
-          code = pr & 0xFFu;
+          o[k >> 2] |= (uint32_t)(pr & 0xFFu) << ((k & 3) * 8);
         }
-        out[k >> 2] |= code << ((k & 3) * 8);
+        out = make_uint2(o[0], o[1]);
       }
-      reinterpret_cast<uint2 *>(p.q)[i] = make_uint2(out[0], out[1]);
+      reinterpret_cast<uint2 *>(p.q)[i] = out;
     }
   }
 }
