@@ -217,24 +217,31 @@ __device__ __forceinline__ uint32_t e2m1_code(float y) {
 }
 
 // Settle the elements whose bracket codes differ (nonzero nibbles of
-// lo ^ hi): the lower candidate magnitude m fixes the boundary T between m
-// and m + 1; the element takes m + 1 above T, m below, the even one of the
-// two on T.  `src` is the block in memory (elements re-read by index).
+// lo ^ hi, elements 8w..8w+7 in word w): the lower candidate magnitude m
+// fixes the boundary T between m and m + 1; the element takes m + 1 above T,
+// m below, the even one of the two on T.  `src` is the block in memory
+// (elements re-read by index).  32-bit words throughout.
 template <typename T>
-__device__ __forceinline__ uint2 settle_codes(const T *src, uint64_t lo, uint64_t hi, float d) {
-  uint64_t m = lo ^ hi;
-  while (m != 0ull) {
-    const int sh = (__ffsll((long long)m) - 1) & ~3;
-    m &= ~(0xFull << sh);
-    const uint32_t cl = (uint32_t)(lo >> sh) & 7u, ch = (uint32_t)(hi >> sh) & 7u;
-    const uint32_t mlow = min(cl, ch);
+__device__ __forceinline__ uint32_t settle_word(const T *src, uint32_t lo, uint32_t hi, float d) {
+  uint32_t m = lo ^ hi;
+  while (m != 0u) {
+    const int sh = (__ffs(m) - 1) & ~3;
+    m &= ~(0xFu << sh);
+    const uint32_t mlow = min((lo >> sh) & 7u, (hi >> sh) & 7u);
     const float xv = to_f32(src[sh >> 2]);
     const int c = quotient_vs(fabsf(xv), d, e2m1_boundary(mlow));
     const uint32_t mag = c > 0 ? mlow + 1u : (c < 0 ? mlow : ((mlow & 1u) ? mlow + 1u : mlow));
-    const uint32_t code = mag | ((__float_as_uint(xv) >> 28) & 8u);
-    lo = (lo & ~(0xFull << sh)) | ((uint64_t)code << sh);
+    lo = (lo & ~(0xFu << sh)) | ((mag | ((__float_as_uint(xv) >> 28) & 8u)) << sh);
   }
-  return make_uint2((uint32_t)lo, (uint32_t)(lo >> 32));
+  return lo;
+}
+
+template <typename T>
+__device__ __forceinline__ uint2 settle_codes(const T *src, uint32_t lo0, uint32_t hi0, uint32_t lo1, uint32_t hi1,
+                                              float d) {
+  if (lo0 != hi0) lo0 = settle_word(src, lo0, hi0, d);
+  if (lo1 != hi1) lo1 = settle_word(src + 8, lo1, hi1, d);
+  return make_uint2(lo0, lo1);
 }
 
 // The whole block by the definition (extreme global scales only).
@@ -277,9 +284,7 @@ __device__ __forceinline__ uint2 encode16(const Block16<T> &b, const EncodeConst
                  lo0, hi0);
   e2m1x8_bracket(b.elem(8), b.elem(9), b.elem(10), b.elem(11), b.elem(12), b.elem(13), b.elem(14), b.elem(15), rlo,
                  rhi, lo1, hi1);
-  if (((lo0 ^ hi0) | (lo1 ^ hi1)) != 0u)
-    return settle_codes(src, (uint64_t)lo0 | ((uint64_t)lo1 << 32), (uint64_t)hi0 | ((uint64_t)hi1 << 32),
-                        __fmul_rn(e4m3_to_f32(s), k.g));
+  if (((lo0 ^ hi0) | (lo1 ^ hi1)) != 0u) return settle_codes(src, lo0, hi0, lo1, hi1, __fmul_rn(e4m3_to_f32(s), k.g));
   return make_uint2(lo0, lo1);
 }
 
@@ -463,8 +468,11 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
   const int64_t atoms_per_rb = p.K >> 6;
   int st = 0;
   uint32_t ph = 0;
+  // (row block, segment) of unit u, advanced by gridDim.x units per step
+  // without a division in the loop
+  const uint32_t step_rb = gridDim.x / nseg, step_seg = gridDim.x - step_rb * nseg;
+  uint32_t rb = blockIdx.x / nseg, seg = blockIdx.x - rb * nseg;
   for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
-    const uint32_t rb = u / nseg, seg = u - rb * nseg;
     if (!mbar_wait_warp(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag)) break;
     const T *sx = reinterpret_cast<const T *>(ring + st * C::STAGE_BYTES) + rsub * C::COLS + cb * 16;
     const int64_t gcol = (int64_t)seg * C::COLS + cb * 16;
@@ -505,6 +513,9 @@ __global__ void __launch_bounds__(QTmaCfg<T>::THREADS, 1)
     }
     if (__any_sync(0xFFFFFFFFu, stop)) break;       // the whole warp leaves together
     if (++st == C::STAGES) { st = 0; ph ^= 1; }
+    rb += step_rb;
+    seg += step_seg;
+    if (seg >= nseg) { seg -= nseg; ++rb; }
   }
   if (loader && *abort_flag) {
     // a wait ran out: let the copies still in flight land before the CTA's
