@@ -221,15 +221,23 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
                                int64_t K, nvfp4_stream_t stream);
 
 /*
- * The decode-shaped layer with the activation quantize inside the GEMM (row
- * a9 of the layer, "quantize in the producer"): one kernel, whose extra warps
- * encode each K stage of x straight into the MMA's operand tiles; the codes
- * are bit-identical to nvfp4_quantize's and y is bit-identical to w4a4_gemm's.
- * For M <= 128 activation rows only (NVFP4_ERR_UNSUPPORTED otherwise, and for
- * shapes whose plan is not the narrow split-K one).  No workspace.  On B200
- * this is slower than w4a4_gemm for the decode configurations (every weight
- * tile's CTAs re-encode the same activation slice), so w4a4_gemm does not use
- * it; it is kept as the in-producer variant of the layer.
+ * The layer with the activation quantize inside the GEMM (row a9 of the
+ * layer, "quantize in the producer"): one kernel, whose extra warps encode
+ * each K stage of x straight into the MMA's operand tiles on the MMA's N side;
+ * the codes are bit-identical to nvfp4_quantize's.  Two shapes are served:
+ *   - decode-shaped products, M <= 128 activation rows (one narrow tile);
+ *   - narrow weights, N <= 128 rows with any M (the GDN gate projections):
+ *     the weight is the 128-row MMA operand and the activation is encoded in
+ *     tiles of 128 rows.
+ * NVFP4_ERR_UNSUPPORTED when M > 128 and N > 128, and when the device offers
+ * no cluster plan for the shape.  No workspace.  y agrees with w4a4_gemm's
+ * within the GEMM tolerance; it is bit-identical on the decode configurations
+ * and on the 4096 x 96 x 5120 gate product (same K split, same reduction
+ * order).  On B200
+ * w4a4_gemm is as fast or faster for these shapes (decode: every weight
+ * tile's CTAs re-encode the same activation slice; gates: 27.7 against
+ * 28.7 us, within the encoder's own throughput), so w4a4_gemm does not use
+ * it; it is kept as the in-producer form of the layer.
  */
 nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
                              const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,

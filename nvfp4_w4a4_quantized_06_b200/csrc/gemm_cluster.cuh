@@ -65,7 +65,9 @@ struct ClusterCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = BN <= 32 ? 8 : (BN <= 64 ? 6 : 4);
   static constexpr int EPI_WARPS = 4;
-  static constexpr int QWARPS = FUSED ? 8 : 0;
+  // activation encoder warps: a 128-row activation tile (the gate
+  // projections' many tokens) needs three times the encoding of a decode tile
+  static constexpr int QWARPS = FUSED ? (BN >= 128 ? 24 : 8) : 0;
   static constexpr int THREADS = 64 + 32 * (EPI_WARPS + QWARPS);
   static constexpr int SF_COLS = 16 + 16 * SFB_ATOMS;
   static constexpr int SFA_COL = BN;
@@ -286,9 +288,13 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
       // scale atoms.  Rows past rows_b and columns past K encode as zeros.
       const int qt = (int)threadIdx.x - 32 * (2 + C::EPI_WARPS);
       constexpr int QT = 32 * C::QWARPS;
+      // blocks of a stage per encoder thread; bf16 blocks are all loaded
+      // before any is encoded (their loads overlap), fp32 ones one at a time
+      constexpr int NB = sizeof(XT) == 2 ? (BN * 16 + QT - 1) / QT : 1;
       griddep_wait();                                     // x and its scale may come from the preceding kernel
       const EncodeConsts kc = encode_consts(p.x_gscale);
       const XT *x = static_cast<const XT *>(p.x);
+      const int row_base = tb * BN;                       // this tile's first activation row
       int st = 0;
       uint32_t ph = 0;
       for (int ks = ks0; ks < ks1; ++ks) {
@@ -297,19 +303,41 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
         uint8_t *sb = sB + st * C::B_BYTES;
         uint8_t *ssf = sSFB + st * C::SFB_BYTES;
 #pragma unroll 1
-        for (int bi = qt; bi < BN * 16; bi += QT) {
-          const int r = bi >> 4, b = bi & 15;
-          const int64_t col = (int64_t)ks * 256 + b * 16;
-          uint2 w = make_uint2(0u, 0u);
-          uint32_t sc = 0u;
-          if (r < p.rows_b && col < p.K) {
-            const XT *src = x + (int64_t)r * p.ld_x + col;
-            Block16<XT> blk;
-            blk.load(src);
-            w = encode16(blk, kc, rcp_tab, src, &sc);
+        for (int bi0 = qt; bi0 < BN * 16; bi0 += NB * QT) {
+          Block16<XT> blk[NB];
+          bool valid[NB];
+#pragma unroll
+          for (int n = 0; n < NB; ++n) {
+            const int bi = bi0 + n * QT;
+            const int r = bi >> 4, b = bi & 15;
+            const int64_t col = (int64_t)ks * 256 + b * 16;
+            valid[n] = bi < BN * 16 && row_base + r < p.rows_b && col < p.K;
+            blk[n].zero();
+            if (valid[n]) blk[n].load(x + (int64_t)(row_base + r) * p.ld_x + col);
           }
-          *reinterpret_cast<uint2 *>(sb + r * 128 + (((b >> 1) ^ (r & 7)) << 4) + (b & 1) * 8) = w;
-          ssf[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)] = (uint8_t)sc;
+          if (ks + 1 < ks1) {
+            // warm the same blocks of the next stage in L2 while these encode
+#pragma unroll
+            for (int n = 0; n < NB; ++n) {
+              const int bi = bi0 + n * QT;
+              const int r = bi >> 4, b = bi & 15;
+              const int64_t col = (int64_t)(ks + 1) * 256 + b * 16;
+              if (bi < BN * 16 && row_base + r < p.rows_b && col < p.K)
+                prefetch_l2(x + (int64_t)(row_base + r) * p.ld_x + col);
+            }
+          }
+#pragma unroll
+          for (int n = 0; n < NB; ++n) {
+            const int bi = bi0 + n * QT;
+            if (bi >= BN * 16) break;
+            const int r = bi >> 4, b = bi & 15;
+            uint2 w = make_uint2(0u, 0u);
+            uint32_t sc = 0u;
+            if (valid[n])
+              w = encode16(blk[n], kc, rcp_tab, x + (int64_t)(row_base + r) * p.ld_x + (int64_t)ks * 256 + b * 16, &sc);
+            *reinterpret_cast<uint2 *>(sb + r * 128 + (((b >> 1) ^ (r & 7)) << 4) + (b & 1) * 8) = w;
+            ssf[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)] = (uint8_t)sc;
+          }
         }
         fence_proxy_async_shared();                      // the tensor core reads the tile through the async proxy
         __syncwarp();

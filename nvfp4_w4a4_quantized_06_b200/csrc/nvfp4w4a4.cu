@@ -51,6 +51,8 @@ struct DeviceState {
   int pair_clusters = 0;                // co-resident CTA pairs of the pair GEMM
   // co-resident clusters of the split-K cluster GEMM, [BN 32/64/128][size 1..8]
   int split_clusters[3][kMaxSplitCluster + 1] = {};
+  // the same for its 128-wide variant with the activation encoded in the kernel
+  int fused128_clusters[kMaxSplitCluster + 1] = {};
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -81,6 +83,8 @@ cudaError_t set_cluster_attrs() {
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32, __nv_bfloat16>, bf);
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_BF16, float>, bf);
   if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_F32, float>, bf);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_GATES, __nv_bfloat16>, bf);
+  if (e == cudaSuccess) e = set_smem(nvfp4_gemm_cluster_kernel<BN, OUT_GATES, float>, bf);
   return e;
 }
 
@@ -94,7 +98,7 @@ cudaError_t set_quant_attrs() {
 }
 
 // How many clusters of `size` CTAs of the split-K GEMM fit on the device at once.
-template <int BN>
+template <int BN, bool FUSED = false>
 int max_split_clusters(int size, int sms) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -103,12 +107,14 @@ int max_split_clusters(int size, int sms) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(size * sms);
-  cfg.blockDim = dim3(ClusterCfg<BN>::THREADS);
-  cfg.dynamicSmemBytes = ClusterCfg<BN>::SMEM_BYTES;
+  cfg.blockDim = dim3(ClusterCfg<BN, FUSED>::THREADS);
+  cfg.dynamicSmemBytes = ClusterCfg<BN, FUSED>::SMEM_BYTES;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, &cfg) != cudaSuccess) n = 0;
+  cudaError_t e = FUSED ? cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_cluster_kernel<BN, OUT_BF16, __nv_bfloat16>, &cfg)
+                        : cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_cluster_kernel<BN, OUT_BF16>, &cfg);
+  if (e != cudaSuccess) n = 0;
   cudaGetLastError();
   return n;
 }
@@ -157,6 +163,7 @@ nvfp4_status device_state(DeviceState **out) {
       d.split_clusters[0][c] = max_split_clusters<32>(c, sms);
       d.split_clusters[1][c] = max_split_clusters<64>(c, sms);
       d.split_clusters[2][c] = max_split_clusters<128>(c, sms);
+      d.fused128_clusters[c] = max_split_clusters<128, true>(c, sms);
     }
     {
       cudaLaunchConfig_t cfg = {};
@@ -382,24 +389,66 @@ cudaError_t launch_cluster(int mode, unsigned grid, int splits, bool pdl, const 
 }
 
 template <int BN, typename XT>
-cudaError_t launch_cluster_fused(bool bf16_out, unsigned grid, int splits, const CUtensorMap &ma,
-                                 const GemmParams &p, cudaStream_t stream) {
+cudaError_t launch_cluster_fused(int mode, unsigned grid, int splits, const CUtensorMap &ma, const GemmParams &p,
+                                 cudaStream_t stream) {
   using C = ClusterCfg<BN, true>;
-  return bf16_out ? launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_BF16, XT>, grid, C::THREADS, C::SMEM_BYTES, stream,
-                              splits, true, ma, ma, p)
-                  : launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_F32, XT>, grid, C::THREADS, C::SMEM_BYTES, stream,
-                              splits, true, ma, ma, p);
+  if (mode == OUT_BF16)
+    return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_BF16, XT>, grid, C::THREADS, C::SMEM_BYTES, stream, splits,
+                     true, ma, ma, p);
+  if (mode == OUT_GATES)
+    return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_GATES, XT>, grid, C::THREADS, C::SMEM_BYTES, stream, splits,
+                     true, ma, ma, p);
+  return launch_ex(nvfp4_gemm_cluster_kernel<BN, OUT_F32, XT>, grid, C::THREADS, C::SMEM_BYTES, stream, splits, true,
+                   ma, ma, p);
 }
 
-// The decode-shaped layer in one kernel: the activation x (M <= 128 rows)
-// is quantized inside the cluster GEMM (row a9).  Returns UNSUPPORTED when the
-// plan is not a cluster plan with the activation on the narrow side.
+// Plan of the one-kernel layer (activation encoded inside the split-K
+// cluster GEMM, on the MMA's N side): decode-shaped products (M <= 128
+// activation rows, one narrow tile) take the two-kernel layer's plan; products
+// with a narrow weight (N <= 128, the gate projections) put the weight on the
+// 128-row side and the activation on the N side in tiles of 128 rows, and
+// split K over the largest cluster that keeps all tiles in one wave.
+// kind SINGLE means there is no such plan.
+Plan fused_plan(int64_t M, int64_t N, int64_t K, const DeviceState &d) {
+  if (M <= 128) {
+    Plan pl = make_plan(M, N, K, d);
+    if (pl.kind != Plan::CLUSTER || !pl.swap) pl.kind = Plan::SINGLE;
+    return pl;
+  }
+  Plan pl{};
+  pl.kind = Plan::SINGLE;
+  if (N > 128) return pl;
+  pl.kstages = (int)((K / 64 + 3) / 4);
+  pl.swap = true;
+  pl.bn = 128;
+  pl.tiles_a = 1;
+  pl.tiles_b = (int)((M + 127) / 128);
+  int best = 0;
+  int64_t best_cost = 0;
+  for (int c = 1; c <= max_splits_for_bn(128) && c <= pl.kstages; ++c) {
+    const int fit = d.fused128_clusters[c];
+    if (fit <= 0) continue;
+    const int64_t waves = (pl.tiles_b + fit - 1) / fit;
+    const int64_t cost = waves * ((pl.kstages + c - 1) / c + 1);
+    if (best == 0 || cost < best_cost) { best = c; best_cost = cost; }
+  }
+  if (best == 0) return pl;
+  pl.kind = Plan::CLUSTER;
+  pl.splits = best;
+  pl.grid = pl.tiles_b * best;
+  return pl;
+}
+
+// The layer in one kernel: the activation x is quantized inside the cluster
+// GEMM (row a9), for decode-shaped products and for narrow weights (the gate
+// projections, optionally with their activations in the epilogue:
+// gates_n_a >= 0).  Returns UNSUPPORTED when there is no such plan.
 nvfp4_status w4a4_fused_impl(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
                              const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
                              nvfp4_out_dtype y_dt, int64_t ld_y, int64_t M, int64_t N, int64_t K,
-                             const DeviceState &dev, cudaStream_t stream) {
-  const Plan pl = make_plan(M, N, K, dev);
-  if (pl.kind != Plan::CLUSTER || !pl.swap) return NVFP4_ERR_UNSUPPORTED;
+                             const DeviceState &dev, cudaStream_t stream, int64_t gates_n_a = -1) {
+  const Plan pl = fused_plan(M, N, K, dev);
+  if (pl.kind != Plan::CLUSTER) return NVFP4_ERR_UNSUPPORTED;
   GemmParams p{};
   p.sfa = w_sf;
   p.ga = x_gscale;
@@ -420,23 +469,25 @@ nvfp4_status w4a4_fused_impl(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, c
   p.x = x;
   p.ld_x = ld_x;
   p.x_gscale = x_gscale;
+  p.n_split = (int)(gates_n_a >= 0 ? gates_n_a : 0);
   CUtensorMap ma;
   if (!make_codes_map(&ma, w_codes, N, K, 128)) return NVFP4_ERR_CUDA;
-  const bool bf = y_dt == NVFP4_OUT_BF16, xb = x_dt == NVFP4_IN_BF16;
+  const int mode = gates_n_a >= 0 ? OUT_GATES : (y_dt == NVFP4_OUT_BF16 ? OUT_BF16 : OUT_F32);
+  const bool xb = x_dt == NVFP4_IN_BF16;
   const unsigned g = (unsigned)pl.grid;
   cudaError_t e;
   switch (pl.bn) {
     case 32:
-      e = xb ? launch_cluster_fused<32, __nv_bfloat16>(bf, g, pl.splits, ma, p, stream)
-             : launch_cluster_fused<32, float>(bf, g, pl.splits, ma, p, stream);
+      e = xb ? launch_cluster_fused<32, __nv_bfloat16>(mode, g, pl.splits, ma, p, stream)
+             : launch_cluster_fused<32, float>(mode, g, pl.splits, ma, p, stream);
       break;
     case 64:
-      e = xb ? launch_cluster_fused<64, __nv_bfloat16>(bf, g, pl.splits, ma, p, stream)
-             : launch_cluster_fused<64, float>(bf, g, pl.splits, ma, p, stream);
+      e = xb ? launch_cluster_fused<64, __nv_bfloat16>(mode, g, pl.splits, ma, p, stream)
+             : launch_cluster_fused<64, float>(mode, g, pl.splits, ma, p, stream);
       break;
     default:
-      e = xb ? launch_cluster_fused<128, __nv_bfloat16>(bf, g, pl.splits, ma, p, stream)
-             : launch_cluster_fused<128, float>(bf, g, pl.splits, ma, p, stream);
+      e = xb ? launch_cluster_fused<128, __nv_bfloat16>(mode, g, pl.splits, ma, p, stream)
+             : launch_cluster_fused<128, float>(mode, g, pl.splits, ma, p, stream);
       break;
   }
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -877,7 +928,7 @@ nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, c
                              nvfp4_stream_t stream) {
   if (x_dt != NVFP4_IN_BF16 && x_dt != NVFP4_IN_F32) return NVFP4_ERR_DTYPE;
   if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ld_x < K) return NVFP4_ERR_SHAPE;
-  if (M > 128) return NVFP4_ERR_UNSUPPORTED;
+  if (M > 128 && N > 128) return NVFP4_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return NVFP4_OK;
   if (!x || !x_gscale) return NVFP4_ERR_NULL;
   const int esz = x_dt == NVFP4_IN_BF16 ? 2 : 4;

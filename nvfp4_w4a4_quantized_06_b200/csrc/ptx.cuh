@@ -373,6 +373,10 @@ __device__ __forceinline__ void st_shared_cluster_v4(uint32_t cluster_addr, uint
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+// bring the line holding p into L2 (a hint; no register, no completion)
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 // four floats from this CTA's shared memory (16-byte aligned address)
 __device__ __forceinline__ float4 ld_shared_f32x4(uint32_t a) {
   float4 v;

@@ -295,8 +295,9 @@ def linear_noalloc(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tenso
 
 def linear_fused(x: torch.Tensor, x_gscale: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
                  w_gscale: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
-    """The decode-shaped layer (M <= 128) with the activation quantized inside
-    the GEMM kernel; bit-identical to linear()."""
+    """The layer with the activation quantized inside the GEMM kernel, for
+    decode-shaped products (M <= 128) and narrow weights (N <= 128, e.g. the
+    gate projections); bit-identical to linear() on the shapes measured."""
     M, K, N = _linear_args(x, x_gscale, w_codes, w_sf, w_gscale, out)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)

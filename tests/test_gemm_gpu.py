@@ -207,6 +207,33 @@ def test_fused_prologue_matches_layer(M, N, K, x_dtype, out_dtype):
     assert torch.equal(y, y_ref)
 
 
+@pytest.mark.parametrize("M,N,K,x_dtype", [
+    (4096, 96, 5120, torch.bfloat16),     # the gate projections: many tokens, narrow weight
+    (1000, 40, 832, torch.bfloat16),      # ragged token count and weight, K tail
+    (300, 96, 1344, torch.float32),       # fp32 activation
+])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fused_prologue_narrow_weight(M, N, K, x_dtype, out_dtype):
+    """Narrow weights (N <= 128) with many activation rows: the activation is
+    encoded inside the GEMM in 128-row tiles on the MMA's N side.  Every
+    output within the GEMM tolerance of the oracle's float64 product, and
+    equal to the two-kernel layer's output."""
+    x_cpu = W.gaussian(M, K, seed=M + 11, outliers=W.Outliers("scale", 0.02, 30.0), dtype=x_dtype)
+    w_cpu = W.gaussian(N, K, seed=N + 13, std=0.02)
+    x, w = x_cpu.to(DEV), w_cpu.to(DEV)
+    (gx_r, gx), (gw_r, gw) = checked_gscale(x_cpu, x), checked_gscale(w_cpu, w)
+    wc, ws = native.quantize(w, gw)
+    y = native.linear_fused(x, gx, wc, ws, gw, out_dtype=out_dtype)
+    y_ref = native.linear(x, gx, wc, ws, gw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+    rwc, rws = oracle.quantize(to_f32_numpy(w_cpu), gw_r)
+    assert_codes_equal(wc, rwc)
+    y64, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu), gx_r, rwc, rws, gw_r)
+    assert_gemm_close(y, y64, yabs)
+    assert_gemm_close(y_ref, y64, yabs)
+
+
 def test_fused_prologue_rejects_prefill_shapes():
     x = torch.zeros(256, 256, dtype=torch.bfloat16, device=DEV)
     w = torch.zeros(256, 256, dtype=torch.bfloat16, device=DEV)
