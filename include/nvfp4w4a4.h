@@ -353,8 +353,8 @@ nvfp4_status nvfp4_harmonize_requant(uint8_t *codes, uint8_t *sf, int64_t rows_t
  *   sf       : nvfp4_sf_bytes(rows, K) bytes (device); padding rows zeroed.
  *   inv_out  : NULL or [rows] floats (device): inv_r.
  * Errors: NVFP4_ERR_SHAPE for eps <= 0 or not finite; NVFP4_ERR_UNSUPPORTED
- * when two rows of x and the weight do not fit in one CTA's shared memory
- * (K above 38592 for bf16 x, 23168 for fp32 x).
+ * when the norm weight does not fit in one CTA's shared memory beside the
+ * encoder's staging (K above 111872).
  */
 nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
                                     const uint16_t *w, int zero_centered, float eps, const float *gscale,

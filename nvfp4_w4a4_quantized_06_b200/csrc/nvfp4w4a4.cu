@@ -93,7 +93,7 @@ constexpr int kSmemOptin = 232448;   // 227 KB, the per-CTA opt-in limit of sm_1
 template <typename T>
 cudaError_t set_quant_attrs() {
   cudaError_t e = set_smem(quantize_tma_kernel<T>, QTmaCfg<T>::SMEM_BYTES);
-  if (e == cudaSuccess) e = set_smem(rmsnorm_quantize_kernel<T>, kSmemOptin);
+  if (e == cudaSuccess) e = set_smem(rmsnorm_quantize_warp_kernel<T>, kSmemOptin);
   return e;
 }
 
@@ -1065,10 +1065,8 @@ nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t ro
   if ((rows > 0 && (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 7))) || (ld_x * esz) % 16 != 0 ||
       !aligned16(sf) || !aligned16(w) || (inv_out && (reinterpret_cast<uintptr_t>(inv_out) & 3)))
     return NVFP4_ERR_ALIGN;
-  int stages = 4;
-  while (stages > 2 && rms_smem_bytes(K, esz, stages) > 56 * 1024) --stages;
-  const int64_t smem = rms_smem_bytes(K, esz, stages);
-  if (smem > kSmemOptin) return NVFP4_ERR_UNSUPPORTED;
+  // the norm weight is staged in one CTA's shared memory
+  if (rms_warp_smem_bytes(K) > kSmemOptin) return NVFP4_ERR_UNSUPPORTED;
   DeviceState *dev = nullptr;
   nvfp4_status st = device_state(&dev);
   if (st != NVFP4_OK) return st;
@@ -1076,21 +1074,24 @@ nvfp4_status nvfp4_rmsnorm_quantize(const void *x, nvfp4_in_dtype dt, int64_t ro
   if (rows == 0 && pad_rows == 0) return NVFP4_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   RmsQuantParams p{x, rows, K, ld_x, reinterpret_cast<const __nv_bfloat16 *>(w), zero_centered ? 1 : 0, eps,
-                   gscale, codes, sf, inv_out, pad_rows, stages, dev->err};
+                   gscale, codes, sf, inv_out, pad_rows};
+  // one warp per row (no CTA barrier per row)
+  const size_t wsmem = (size_t)rms_warp_smem_bytes(K);
   int per_sm = 0;
   cudaError_t e = dt == NVFP4_IN_BF16
-                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quantize_kernel<__nv_bfloat16>,
-                                                                      kRmsThreads, (size_t)smem)
-                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quantize_kernel<float>,
-                                                                      kRmsThreads, (size_t)smem);
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quantize_warp_kernel<__nv_bfloat16>,
+                                                                      kRmsWarpThreads, wsmem)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rmsnorm_quantize_warp_kernel<float>,
+                                                                      kRmsWarpThreads, wsmem);
   if (e != cudaSuccess || per_sm < 1) return NVFP4_ERR_CUDA;
   int64_t grid = (int64_t)per_sm * dev->sms;
-  if (grid > rows) grid = rows;
+  const int64_t need = (rows + kRmsWarpThreads / 32 - 1) / (kRmsWarpThreads / 32);
+  if (grid > need) grid = need;
   if (grid < 1) grid = 1;
   e = dt == NVFP4_IN_BF16
-          ? launch_ex(rmsnorm_quantize_kernel<__nv_bfloat16>, (unsigned)grid, (unsigned)kRmsThreads, (size_t)smem, s, 0,
-                      false, p)
-          : launch_ex(rmsnorm_quantize_kernel<float>, (unsigned)grid, (unsigned)kRmsThreads, (size_t)smem, s, 0, false,
+          ? launch_ex(rmsnorm_quantize_warp_kernel<__nv_bfloat16>, (unsigned)grid, (unsigned)kRmsWarpThreads, wsmem, s,
+                      0, false, p)
+          : launch_ex(rmsnorm_quantize_warp_kernel<float>, (unsigned)grid, (unsigned)kRmsWarpThreads, wsmem, s, 0, false,
                       p);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   return launched();

@@ -925,15 +925,6 @@ __global__ void __launch_bounds__(256) harmonize_requant_kernel(HarmonizeParams 
 // eps, and rsqrt (at most one ulp) gives 1/sqrt to ~2^-48: the fp32 rounding
 // then agrees with the exact one except when the exact value lies within
 // that distance of a midpoint between two floats.
-//
-// One CTA of 256 threads per row at a time, persistent over rows
-// blockIdx.x + j * gridDim.x; each row arrives whole in a ring slot by a
-// contiguous bulk copy.  Thread t owns blocks t, t + 256, ... of the row:
-// phase 1 sums their squares (warp shuffles, then one fp64 per warp in
-// shared memory and a CTA barrier), phase 2 writes y back over x in the
-// slot (the encoder's settling path re-reads it) and encodes it.  The slot
-// of row j - 1 is refilled with row j - 1 + STAGES right after the barrier
-// of row j, when every thread is done with it.
 struct RmsQuantParams {
   const void *x;
   int64_t rows, K, ld_x;
@@ -945,104 +936,59 @@ struct RmsQuantParams {
   uint8_t *sf;
   float *inv_out;           // per-row factor [rows], or null
   int64_t pad_rows;
-  int stages;
-  unsigned *err;
 };
 
-constexpr int kRmsThreads = 256;
+// The same RMSNorm-fused quantize with one warp per row: lane l owns blocks
+// l, l + 32, ... of its row.  Phase 1 sums their squares in fp64 and the warp
+// reduces the sum with shuffles (no CTA barrier); phase 2 reads the blocks
+// again (from L2), forms y and encodes it.  Each lane keeps its current block
+// of y in a 32-byte shared slot, where the encoder's settling path re-reads
+// elements.  The norm weight is staged once per CTA.
+constexpr int kRmsWarpThreads = 256;
 
-// shared memory of the kernel: ring, norm weight, barriers, warp sums, rcp table, abort flag
-__host__ __device__ constexpr int64_t rms_smem_bytes(int64_t K, int esz, int stages) {
-  return stages * K * esz + K * 2 + stages * 8 + 2 * (kRmsThreads / 32) * 8 + 128 * 4 + 16;
+__host__ __device__ constexpr int64_t rms_warp_smem_bytes(int64_t K) {
+  return K * 2 + kRmsWarpThreads * 32 + 128 * 4;
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kRmsThreads, 4) rmsnorm_quantize_kernel(const RmsQuantParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int stages = p.stages;
-  const uint32_t row_bytes = (uint32_t)(p.K * (int64_t)sizeof(T));
-  uint8_t *ring = smem;
-  const uint32_t *wsm = reinterpret_cast<const uint32_t *>(ring + (size_t)stages * row_bytes);
-  uint64_t *full = reinterpret_cast<uint64_t *>(ring + (size_t)stages * row_bytes + p.K * 2);
-  double *red = reinterpret_cast<double *>(full + stages);
-  float *rcp_tab = reinterpret_cast<float *>(red + 2 * (kRmsThreads / 32));
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(rcp_tab + 128);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const T *x = static_cast<const T *>(p.x);
-  auto issue = [&](int st, int64_t row) {
-    mbar_arrive_expect_tx(&full[st], row_bytes);
-    bulk_load(ring + (size_t)st * row_bytes, x + row * p.ld_x, row_bytes, &full[st]);
-  };
-  if (tid == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
+__global__ void __launch_bounds__(kRmsWarpThreads, 4) rmsnorm_quantize_warp_kernel(const RmsQuantParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __nv_bfloat16 *wsm = reinterpret_cast<__nv_bfloat16 *>(smem);
+  __nv_bfloat16 *ystage = reinterpret_cast<__nv_bfloat16 *>(smem + p.K * 2) + threadIdx.x * 16;
+  float *rcp_tab = reinterpret_cast<float *>(smem + p.K * 2 + kRmsWarpThreads * 32);
   fill_rcp_table(rcp_tab);
   pdl_prologue();
-  for (int64_t i = tid; i < (p.K >> 3); i += kRmsThreads)
-    reinterpret_cast<uint4 *>(const_cast<uint32_t *>(wsm))[i] = __ldg(reinterpret_cast<const uint4 *>(p.w) + i);
+  for (int64_t i = threadIdx.x; i < (p.K >> 3); i += kRmsWarpThreads)
+    reinterpret_cast<uint4 *>(wsm)[i] = __ldg(reinterpret_cast<const uint4 *>(p.w) + i);
   __syncthreads();
-  int64_t issued = 0;   // rows of this CTA handed to the copy engine (thread 0's count)
-  if (tid == 0)
-    for (int s = 0; s < stages; ++s) {
-      const int64_t row = blockIdx.x + (int64_t)s * gridDim.x;
-      if (row >= p.rows) break;
-      issue(s, row);
-      ++issued;
-    }
-
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (kRmsWarpThreads / 32);
+  const T *x = static_cast<const T *>(p.x);
   const EncodeConsts kc = encode_consts(p.gscale);
   const int nb = (int)(p.K >> 4);
   const double rk = __drcp_rn((double)p.K);
   const double eps = (double)p.eps;
-  int st = 0;
-  uint32_t ph = 0;
-  int64_t j = 0;
-  bool stopped = false;
-  for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x, ++j) {
-    const bool ok = mbar_wait(&full[st], ph, p.err, ERR_EPILOGUE, abort_flag);
-    T *sx = reinterpret_cast<T *>(ring + (size_t)st * row_bytes);
+  for (int64_t row = (int64_t)blockIdx.x * (kRmsWarpThreads / 32) + (threadIdx.x >> 5); row < p.rows; row += nwarps) {
+    const T *xr = x + row * p.ld_x;
     double acc = 0.0;
-    if (ok) {
-      for (int c = tid; c < nb; c += kRmsThreads) {
-        Block16<T> b;
-        b.load_shared(sx + c * 16);
+#pragma unroll 2
+    for (int c = lane; c < nb; c += 32) {
+      Block16<T> b;
+      b.load(xr + c * 16);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const double v = (double)b.elem(e);
-          acc = fma(v, v, acc);
-        }
+      for (int e = 0; e < 16; ++e) {
+        const double v = (double)b.elem(e);
+        acc = fma(v, v, acc);
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    double *rw = red + (j & 1) * (kRmsThreads / 32);
-    if (lane == 0) rw[warp] = acc;
-    if (__syncthreads_or(!ok)) {      // a wait ran out: the whole CTA stops here
-      stopped = true;
-      break;
-    }
-    // every thread is done with row j - 1: its slot takes row j - 1 + stages
-    if (tid == 0 && j >= 1) {
-      const int64_t nr = blockIdx.x + (j - 1 + stages) * (int64_t)gridDim.x;
-      if (nr < p.rows) {
-        issue((int)((j - 1) % stages), nr);
-        ++issued;
-      }
-    }
-    double ssq = 0.0;
-#pragma unroll
-    for (int w = 0; w < kRmsThreads / 32; ++w) ssq += rw[w];
-    const float inv = __double2float_rn(rsqrt(fma(ssq, rk, eps)));
-    if (tid == 0 && p.inv_out) p.inv_out[row] = inv;
-
+    const float inv = __double2float_rn(rsqrt(fma(acc, rk, eps)));
+    if (lane == 0 && p.inv_out) p.inv_out[row] = inv;
     uint8_t *crow = p.codes + row * (p.K >> 1);
-    for (int c = tid; c < nb; c += kRmsThreads) {
+    for (int c = lane; c < nb; c += 32) {
       Block16<T> xb;
-      xb.load_shared(sx + c * 16);
-      __nv_bfloat16 *ysrc = reinterpret_cast<__nv_bfloat16 *>(sx + c * 16);
+      xb.load(xr + c * 16);
       const uint4 w0 = reinterpret_cast<const uint4 *>(wsm)[2 * c], w1 = reinterpret_cast<const uint4 *>(wsm)[2 * c + 1];
       const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       Block16<__nv_bfloat16> yb;
@@ -1058,26 +1004,13 @@ __global__ void __launch_bounds__(kRmsThreads, 4) rmsnorm_quantize_kernel(const 
         __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
         yb.w[i] = *reinterpret_cast<uint32_t *>(&h);
       }
-      reinterpret_cast<uint4 *>(ysrc)[0] = make_uint4(yb.w[0], yb.w[1], yb.w[2], yb.w[3]);
-      reinterpret_cast<uint4 *>(ysrc)[1] = make_uint4(yb.w[4], yb.w[5], yb.w[6], yb.w[7]);
+      reinterpret_cast<uint4 *>(ystage)[0] = make_uint4(yb.w[0], yb.w[1], yb.w[2], yb.w[3]);
+      reinterpret_cast<uint4 *>(ystage)[1] = make_uint4(yb.w[4], yb.w[5], yb.w[6], yb.w[7]);
       uint32_t s;
-      const uint2 word = encode16(yb, kc, rcp_tab, ysrc, &s);
+      const uint2 word = encode16(yb, kc, rcp_tab, ystage, &s);
       *reinterpret_cast<uint2 *>(crow + c * 8) = word;
       p.sf[sf_index(row, c, p.K)] = static_cast<uint8_t>(s);
     }
-    fence_proxy_async_shared();       // y was written through the generic proxy; the next copy overwrites it
-    if (++st == stages) {
-      st = 0;
-      ph ^= 1;
-    }
-  }
-  if (stopped) {
-    // let the copies still in flight land before the CTA's memory goes away
-    if (tid == 0) {
-      volatile int never = 0;
-      for (int64_t k = j; k < issued; ++k) mbar_wait(&full[k % stages], (uint32_t)((k / stages) & 1), p.err, ERR_EPILOGUE, &never);
-    }
-    return;
   }
   zero_pad_scales(p.sf, p.rows, p.pad_rows, p.K);
 }

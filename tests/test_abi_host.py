@@ -134,11 +134,11 @@ def test_requant_and_rmsnorm_validation(L):
     assert r(FAKE, 0, 4, 256, 256, None, 0, 1e-6, *tail) == 1               # null weight
     assert r(FAKE, 0, 4, 256, 256, FAKE + 8, 0, 1e-6, *tail) == 3           # misaligned weight
     assert r(FAKE, 0, 4, 256, 256, FAKE, 0, 1e-6, FAKE, FAKE, FAKE, FAKE + 2, None) == 3   # misaligned inv
-    # two rows and the weight must fit in one CTA's shared memory
-    assert r(FAKE, 0, 4, 38656, 38656, FAKE, 0, 1e-6, *tail) == 5
-    assert r(FAKE, 1, 4, 23232, 23232, FAKE, 0, 1e-6, *tail) == 5
-    assert r(FAKE, 0, 4, 38592, 38592, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
-    assert r(FAKE, 1, 4, 23168, 23168, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
+    # the norm weight must fit in one CTA's shared memory beside the staging
+    assert r(FAKE, 0, 4, 111936, 111936, FAKE, 0, 1e-6, *tail) == 5
+    assert r(FAKE, 1, 4, 111936, 111936, FAKE, 0, 1e-6, *tail) == 5
+    assert r(FAKE, 0, 4, 111872, 111872, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
+    assert r(FAKE, 1, 4, 111872, 111872, FAKE, 0, 1e-6, *tail) not in (2, 3, 5)
 
 
 def test_error_word_bits_match_the_header(L):
