@@ -18,7 +18,16 @@
 // 2.43 ms when the MMA thread issued tcgen05.cp.cta_group::2 per K block),
 // while eight "scale warps" (per TMEM lane quarter one for the A scales and
 // one for the B scales) store them from registers at several hundred B/clk
-// and leave the single MMA-issuing thread nothing but MMAs.
+// and leave the single MMA-issuing thread nothing but MMAs.  Issuing the
+// copies one stage ahead of the MMAs does not help either (4.03 ms): the
+// copies and the MMAs share the tensor pipe.  What the scale path still
+// costs (about 0.37 ms of the 2.45 ms prefill product) is mostly the shared
+// memory reads of the replicated B scales: every lane quarter must hold all
+// 256 B-row scales, so four warps each read the same 4 KB per stage; letting
+// three of them skip the reads (wrong results, timing only) gives 2.24 ms.
+// Each quarter's MMA reads only its own word of the A atom (rows 32q + l),
+// but the atom's layout puts those words 16 bytes apart, so reading only
+// them takes the same number of shared-memory wavefronts.
 //
 // BF16 output leaves through TMA stores: each epilogue warp drains its
 // accumulator columns, hands TMEM back, converts to BF16 in a 32 x 32 staging
