@@ -357,6 +357,9 @@ def measure_secondary(native, dev, only=None):
         times = []
         for i in range(reps):
             flush.zero_()
+            # keep the GPU busy while the host enqueues the start event and
+            # the call, so that host-side call overhead is not timed as GPU time
+            torch.cuda._sleep(100000)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             fn()

@@ -290,9 +290,12 @@ nvfp4_status w4a4_gdn_gates(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, co
  *              FP32 output is the exact value rounded once to fp32, BF16 output
  *              is that fp32 value rounded to bf16.
  *   err_stats: NULL or 2 doubles (device, 8-byte aligned), overwritten with
- *              [sum of (x - out)^2 in float64, sum of x^2]; the relative error
- *              is sqrt(err_stats[0] / err_stats[1]).  The sums are accumulated
- *              with atomics, so their rounding depends on timing (float64).
+ *              [sum of (x - q)^2, sum of x^2], q the exact NVFP4 value of x;
+ *              the relative error is sqrt(err_stats[0] / err_stats[1]).  Each
+ *              16-element block is summed in fp32 and the blocks in float64,
+ *              so each sum is within a relative 18 * 2^-24 (about 1.1e-6) of
+ *              the exact one; the blocks are added with atomics, so the last
+ *              bits depend on timing.
  * Preconditions: K % 64 == 0; 16-byte aligned pointers and row strides.
  */
 nvfp4_status nvfp4_fake_quant(const void *x, nvfp4_in_dtype dt, int64_t rows, int64_t K, int64_t ld_x,

@@ -592,9 +592,18 @@ __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16 *dst, const
 // Every element replaced by the NVFP4 value it quantizes to (the same
 // encoder as the quantize kernels, then dec(q) * dec(s) * g: the first
 // product is exact, so the result is fl32 of the exact value), plus the
-// float64 sums of the squared error against the exact value and of the
-// squared input.  One warp per 512-column
-// row segment, lane l owning block l, like quantize_rows_kernel.
+// sums of the squared error against the exact value and of the squared
+// input.  One warp per 512-column row segment, lane l owning block l, like
+// quantize_rows_kernel.
+// The sums are taken in fp32 over each 16-element block and in float64
+// across blocks, so that no element needs a float64 conversion (those ran
+// on the conversion pipe, which set the kernel's time).  The error of an
+// element, x - q with q = dec(q)*dec(s)*g, is formed from p = fl32(q) and
+// its remainder r = q - p (one FMA, exact): x - p is exact wherever q is
+// non-zero and unsaturated (x and p within a factor of two), so d = x - p - r
+// carries one rounding.  A block's sums of non-negative fp32 terms then
+// carry a relative error below 18 * 2^-24 (about 1.1e-6); the float64 sum
+// across blocks adds nothing visible at that level.
 template <typename T, typename OUT>
 __global__ void __launch_bounds__(256, 4) fake_quant_kernel(FakeQuantParams p) {
   __shared__ float rcp_tab[128];
@@ -638,15 +647,19 @@ __global__ void __launch_bounds__(256, 4) fake_quant_kernel(FakeQuantParams p) {
     float qv[16];
     e2m1x16_times_scale(w, e4m3_to_f32(s), qv);
     float v[16];
+    float se_b = 0.0f, sx_b = 0.0f;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const float qs = qv[e];
-      v[e] = __fmul_rn(qs, kc.g);
-      // the error is taken against the exact NVFP4 value (exact in float64)
-      const double xe = (double)b.elem(e), d = xe - (double)qs * (double)kc.g;
-      se = fma(d, d, se);
-      sx = fma(xe, xe, sx);
+      const float pv = __fmul_rn(qs, kc.g);
+      v[e] = pv;
+      const float xe = b.elem(e);
+      const float d = __fsub_rn(__fsub_rn(xe, pv), __fmaf_rn(qs, kc.g, -pv));
+      se_b = __fmaf_rn(d, d, se_b);
+      sx_b = __fmaf_rn(xe, xe, sx_b);
     }
+    se += (double)se_b;
+    sx += (double)sx_b;
     store16<OUT>(out + row * p.ld_out + col, v);
     }
   }
