@@ -90,7 +90,19 @@ def _flow_main(rank: int, world: int, port: int, q):
         class Stream:
             cuda_stream = 0
 
+            def __init__(self, *a, **k):
+                pass
+
+            def wait_stream(self, other):
+                pass
+
+            def wait_event(self, ev):
+                pass
+
+        import contextlib
         torch.cuda.Event = Ev
+        torch.cuda.Stream = Stream
+        torch.cuda.stream = lambda s: contextlib.nullcontext()
         torch.cuda.synchronize = lambda *a, **k: None
         torch.cuda.current_stream = lambda *a, **k: Stream()
         torch.cuda.empty_cache = lambda: None
