@@ -721,17 +721,23 @@ __device__ __forceinline__ uint2 fp8x8(const float (&v)[8], float s, float rlo, 
     lo[w] = (uint32_t)l0 | ((uint32_t)l1 << 16);
     hi[w] = (uint32_t)h0 | ((uint32_t)h1 << 16);
   }
-  const uint32_t d0 = lo[0] ^ hi[0], d1 = lo[1] ^ hi[1];
-  if ((d0 | d1) != 0u) {
+  // differing bytes are settled one per lane per round: the warp runs as
+  // many rounds as its lane with the most of them (mostly one), not one
+  // round per byte position that any lane has
+  uint32_t d0 = lo[0] ^ hi[0], d1 = lo[1] ^ hi[1];
+  while ((d0 | d1) != 0u) {
+    const bool w = d0 == 0u;
+    const uint32_t d = w ? d1 : d0;
+    const int sh = (__ffs(d) - 1) & ~7;
+    const int k = (w ? 4 : 0) + (sh >> 3);
+    if (w) d1 &= ~(0xFFu << sh); else d0 &= ~(0xFFu << sh);
+    float xv = v[0];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t dk = (k < 4 ? d0 : d1) >> ((k & 3) * 8) & 0xFFu;
-      if (dk != 0u) {
-        const int w = k >> 2, sh = (k & 3) * 8;
-        const uint32_t code = fp8_settle(v[k], s, lo[w] >> sh & 0xFFu, hi[w] >> sh & 0xFFu, mid_tab);
-        lo[w] = (lo[w] & ~(0xFFu << sh)) | (code << sh);
-      }
-    }
+    for (int j = 1; j < 8; ++j) xv = k == j ? v[j] : xv;
+    const uint32_t lw = w ? lo[1] : lo[0], hw = w ? hi[1] : hi[0];
+    const uint32_t code = fp8_settle(xv, s, lw >> sh & 0xFFu, hw >> sh & 0xFFu, mid_tab);
+    const uint32_t nw = (lw & ~(0xFFu << sh)) | (code << sh);
+    if (w) lo[1] = nw; else lo[0] = nw;
   }
   return make_uint2(lo[0], lo[1]);
 }
