@@ -43,12 +43,12 @@ namespace nvfp4 {
 // "前提2"): a goes through softplus and the exponential, alpha = exp(-softplus(a))
 // (the share of the state that is kept), b through the logistic sigmoid,
 // beta = 1 / (1 + exp(-b)).  The model's per-head decay scale and bias are
-// not part of this layer (unit scale, zero bias).  CUDA's expf / log1pf.
-__device__ __forceinline__ float gate_keep(float a) {
-  const float sp = a > 0.0f ? a + log1pf(expf(-a)) : log1pf(expf(a));
-  return expf(-sp);
-}
-__device__ __forceinline__ float gate_write(float b) { return 1.0f / (1.0f + expf(-b)); }
+// not part of this layer (unit scale, zero bias).  Since
+// exp(-softplus(a)) = exp(-log(1 + e^a)) = 1 / (1 + e^a), both take one CUDA
+// expf, one add and one correctly rounded reciprocal (a few ulp in all; an
+// overflowing exponential gives the limit 0).
+__device__ __forceinline__ float gate_keep(float a) { return __frcp_rn(__fadd_rn(1.0f, expf(a))); }
+__device__ __forceinline__ float gate_write(float b) { return __frcp_rn(__fadd_rn(1.0f, expf(-b))); }
 
 // FUSED: the activation (the B operand of decode-shaped products) is read
 // as bf16/fp32 and quantized inside the kernel by QWARPS extra warps, which
