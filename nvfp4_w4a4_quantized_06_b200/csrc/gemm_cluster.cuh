@@ -194,7 +194,12 @@ __global__ void __launch_bounds__(ClusterCfg<BN, !std::is_void<XT>::value>::THRE
     fence_barrier_init();
     // the first ring's worth of the operand that does not depend on the
     // preceding kernel streams in from here on, while the rest of the CTA
-    // sets up (TMEM, tables) and before the preceding kernel has finished
+    // sets up (TMEM, tables) and before the preceding kernel has finished.
+    // That holds where the preceding kernel is this library's activation
+    // quantize, which lets this grid start only after everything before it
+    // has completed.  The fused form follows whatever the caller ran last,
+    // which may still be writing the weight: it waits first.
+    if constexpr (FUSED) griddep_wait();
     for (int i = 0; i < pre; ++i) {
       mbar_arrive_expect_tx(&full[i], stage_bytes(ks0 + i));
       if (a_first) load_a(i, ks0 + i); else load_b(i, ks0 + i);

@@ -234,6 +234,34 @@ def test_fused_prologue_narrow_weight(M, N, K, x_dtype, out_dtype):
     assert_gemm_close(y_ref, y64, yabs)
 
 
+@pytest.mark.parametrize("M,N,K", [(32, 5120, 5120), (4096, 96, 5120)])
+def test_fused_prologue_waits_for_the_weight_writer(M, N, K):
+    """The fused form is launched so that it may start before the previous
+    kernel on the stream has finished.  When that kernel is still writing the
+    weight (here the weight's own quantize, enqueued right before it into a
+    buffer that holds other codes), the product must still see the new
+    weight: every round equals the two-kernel layer run after a full sync."""
+    x_cpu = W.gaussian(M, K, seed=M + 71, outliers=W.Outliers("scale", 0.02, 30.0))
+    w_cpu = W.gaussian(N, K, seed=N + 73, std=0.02)
+    x, w = x_cpu.to(DEV), w_cpu.to(DEV)
+    (_, gx), (_, gw) = checked_gscale(x_cpu, x), checked_gscale(w_cpu, w)
+    wc = torch.empty((N, K // 2), dtype=torch.uint8, device=DEV)
+    ws = torch.empty(native.sf_bytes(N, K), dtype=torch.uint8, device=DEV)
+    native.quantize(w, gw, codes=wc, sf=ws)
+    torch.cuda.synchronize()
+    y_ref = native.linear(x, gx, wc, ws, gw)
+    torch.cuda.synchronize()
+    for fill in (0x77, 0x11, 0xEE, 0x3C):
+        wc.fill_(fill)
+        ws.fill_(0x38)                       # every block scale 1.0
+        torch.cuda.synchronize()
+        native.quantize(w, gw, codes=wc, sf=ws)
+        y = native.linear_fused(x, gx, wc, ws, gw)
+        torch.cuda.synchronize()
+        assert native.last_device_status() == 0
+        assert torch.equal(y, y_ref), fill
+
+
 def test_fused_prologue_rejects_prefill_shapes():
     x = torch.zeros(256, 256, dtype=torch.bfloat16, device=DEV)
     w = torch.zeros(256, 256, dtype=torch.bfloat16, device=DEV)
