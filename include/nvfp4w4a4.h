@@ -235,9 +235,11 @@ nvfp4_status w4a4_gemm_noalloc(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x,
  * and on the 4096 x 96 x 5120 gate product (same K split, same reduction
  * order).  On B200
  * w4a4_gemm is as fast or faster for these shapes (decode: every weight
- * tile's CTAs re-encode the same activation slice; gates: 27.7 against
- * 28.7 us, within the encoder's own throughput), so w4a4_gemm does not use
- * it; it is kept as the in-producer form of the layer.
+ * tile's CTAs re-encode the same activation slice; gates: both about
+ * 27.7 us, the encoder's own throughput), so w4a4_gemm does not use it; it
+ * is kept as the in-producer form of the layer.  It may start before the
+ * stream's preceding work has finished (programmatic launch) but reads
+ * nothing, the weight included, until that work has completed.
  */
 nvfp4_status w4a4_gemm_fused(const void *x, nvfp4_in_dtype x_dt, int64_t ld_x, const float *x_gscale,
                              const uint8_t *w_codes, const uint8_t *w_sf, const float *w_gscale, void *y,
