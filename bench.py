@@ -401,6 +401,14 @@ def measure_secondary(native, dev, only=None):
         res[name] = {"shape": f"{wl.M}x{wl.N}x{wl.K}", "ms": round(ms, 4),
                      "tflops": round(wl.flops / (ms * 1e-3) / 1e12, 1), **hbm(byts, ms),
                      "l2": "512 MB flush between reps"}
+        if name == "gdn_gates_ab":
+            # the W4A4 product against the unquantized one (float64, untimed):
+            # the pages put 4-bit GEMM error on real gate inputs at 8.5-11%
+            w64 = torch.cat([W.make_w(wl, m) for m in range(len(wl.modules))]).to(dev).double()
+            y32 = native.linear(x, gx, wc, wsf, gw, out_dtype=torch.float32, workspace=ws).double()
+            y64 = x.double() @ w64.T
+            res[name]["gemm_rel_error"] = round(float((y32 - y64).norm() / y64.norm()), 5)
+            del w64, y32, y64
         del x, wc, wsf, y, ws
     for name in ("decode_out_proj", "decode_down_proj"):
         if not want(name):

@@ -234,6 +234,22 @@ def test_fused_prologue_narrow_weight(M, N, K, x_dtype, out_dtype):
     assert_gemm_close(y_ref, y64, yabs)
 
 
+def test_gate_product_error_band():
+    """Plausibility, not parity: the W4A4 gate product's relative error against
+    the unquantized float64 product sits near the 4-bit band the pages report
+    for GEMM pre-activations on real gate inputs (8.5-11%, arxiv-wiki page,
+    "주요 결과" (ii)); on these synthetic inputs the oracle's product gives 11.3%."""
+    wl = W.WORKLOADS["gdn_gates_ab"]
+    x = W.make_x(wl).to(DEV)
+    wc, ws, gw, _, _ = _quantized_weight(wl)
+    _, gx = checked_gscale(x.cpu(), x)
+    y = native.linear(x, gx, wc, ws, gw, out_dtype=torch.float32).double()
+    w64 = torch.cat([W.make_w(wl, m) for m in range(len(wl.modules))]).to(DEV).double()
+    y64 = x.double() @ w64.T
+    rel = float((y - y64).norm() / y64.norm())
+    assert 0.07 < rel < 0.15, rel
+
+
 @pytest.mark.parametrize("M,N,K", [(32, 5120, 5120), (4096, 96, 5120)])
 def test_fused_prologue_waits_for_the_weight_writer(M, N, K):
     """The fused form is launched so that it may start before the previous
