@@ -110,8 +110,17 @@ def _flow_main(rank: int, world: int, port: int, q):
         args = types.SimpleNamespace(gpus=world, steps=3, warmup=3, impl="native", workload="decode_out_proj",
                                      headline_only=True, no_cpu_baseline=True, no_e2e=False, oracle_table=False)
         out = bench.run_native(args, rank, world, torch.device("cpu"))
+        # the JSON line's contract: every key the benchmark promises is there
+        missing = [k for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                               "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                               "roofline", "roofline_quant", "e2e", "gpu_launches", "clocks") if k not in out]
+        missing += ["roofline." + k for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")
+                    if k not in out["roofline"]]
+        missing += ["e2e." + k for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")
+                    if k not in out["e2e"]]
+        missing += ["config.workload"] if "workload" not in out["config"] else []
         q.put((rank, out["n_gpus"], out["ms_per_step"], out["value"], out["e2e"]["ms_per_step"],
-               out["config"]["parallelism"]))
+               out["config"]["parallelism"], missing))
     finally:
         dist.destroy_process_group()
 
@@ -128,7 +137,8 @@ def test_benchmark_flow_on_two_gloo_ranks():
         p.join(timeout=60)
         assert p.exitcode == 0
     wl = bench.W.WORKLOADS["decode_out_proj"]
-    for rank, n, ms, value, e2e_ms, par in res:
+    for rank, n, ms, value, e2e_ms, par, missing in res:
+        assert not missing, missing
         assert n == 2 and par == "replicas x2"
         assert ms == pytest.approx(2.0 / 3, rel=1e-3)         # the slower rank's 2 ms over 3 steps
         assert value == pytest.approx(bench.job_throughput(wl.flops, 2, ms), rel=1e-2)
