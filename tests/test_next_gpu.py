@@ -242,9 +242,11 @@ def _check_rmsnorm(x_cpu, w_cpu, eps, zero_centered, rows=None):
     (33, 320, torch.bfloat16, True),
     (300, 5120, torch.bfloat16, False),
     (129, 2048, torch.float32, False),
-    (4096, 5120, torch.bfloat16, True),       # several rows per CTA: the ring refills
+    (4096, 5120, torch.bfloat16, True),       # several rows per warp
     (2000, 1024, torch.float32, True),
-    (64, 17408, torch.bfloat16, False),       # two stages
+    (64, 17408, torch.bfloat16, False),       # 34 blocks per lane
+    (3, 111872, torch.bfloat16, False),       # the widest row the norm weight's shared copy allows
+    (2, 111872, torch.float32, True),
 ])
 def test_rmsnorm_quantize_matches_oracle(rows, K, dtype, zc):
     x = W.gaussian(rows, K, seed=rows + K, outliers=W.Outliers("scale", 0.01, 30.0), dtype=dtype)
