@@ -44,7 +44,7 @@ def test_gdn_gates_fused_epilogue(M):
     """alpha = exp(-softplus(a)) on the 48 a columns, beta = sigmoid(b) on the
     48 b columns, every output of the launch checked.  Both activations have slope at most 1/4, so the bound is a
     quarter of the GEMM's 1e-3 * sum|products|, plus the fp32 evaluation of
-    exp / log1p (a few ulps of values <= 1)."""
+    1 / (1 + e^{+-y}) (a few ulps of values <= 1)."""
     wl = W.WORKLOADS["gdn_gates_ab"]
     codes, sf, gw, rcodes, rsf, rg = _gate_weights(wl)
     x_cpu = W.make_x(wl)[:M]
@@ -60,6 +60,33 @@ def test_gdn_gates_fused_epilogue(M):
     err = np.abs(got - ref)
     assert np.all(err <= tol), float((err - tol).max())
     assert np.all((got >= 0) & (got <= 1))
+
+
+def test_gdn_gates_saturate():
+    """Pre-activations far past where an fp32 exponential overflows (|y| up
+    to about 770): the gates reach their limits 0 and 1, never NaN, and match
+    the oracle's float64 activations within the same bound."""
+    M, N, n_a, K = 64, 96, 48, 256
+    c = torch.linspace(-2.0, 2.0, M).to(torch.bfloat16)
+    t = torch.tensor([((j % 12) + 1) / 8.0 * (1 if j % 2 else -1) for j in range(N)]).to(torch.bfloat16)
+    x_cpu = c[:, None].expand(M, K).contiguous()
+    w_cpu = t[:, None].expand(N, K).contiguous()
+    x, w = x_cpu.to(DEV), w_cpu.to(DEV)
+    (gx_r, gx), (gw_r, gw) = checked_gscale(x_cpu, x), checked_gscale(w_cpu, w)
+    wc, ws = native.quantize(w, gw)
+    out = native.gdn_gates(x, gx, wc, ws, gw, n_a=n_a)
+    torch.cuda.synchronize()
+    assert native.last_device_status() == 0
+    rwc, rws = oracle.quantize(to_f32_numpy(w_cpu), gw_r)
+    y_ref, yabs, _, _ = oracle.linear_reference(to_f32_numpy(x_cpu), gx_r, rwc, rws, gw_r)
+    assert np.abs(y_ref).max() > 600
+    ref = oracle.gdn_gates(y_ref, n_a)
+    got = out.double().cpu().numpy()
+    assert not np.isnan(got).any()
+    tol = 0.25 * GEMM_RTOL * yabs + 1e-5 * np.abs(ref) + 1e-7
+    assert np.all(np.abs(got - ref) <= tol), float((np.abs(got - ref) - tol).max())
+    assert np.all((got >= 0) & (got <= 1))
+    assert (got == 0).any() and (got == 1).any()
 
 
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
